@@ -1,0 +1,462 @@
+"""Benchmark of the paged split-KV decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa|long|mixed|mla|tiny]
+                    [--impl ours|reference]
+
+One step = one paged decode call (partition pass + LSE merge pass) over the
+workload's whole batch, inputs resident in HBM.  The L2 is flushed between
+timed steps (a 512 MiB write, then a 512 MiB read of another buffer so that no
+dirty lines are left to write back during the timed call); each step is timed
+with CUDA events on the launching stream and the per-step times are summed.
+Metric: effective KV-read GB/s = algorithmic KV bytes (every live K/V element
+once) / step time; ms_per_step is the mean step time.
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch of
+independent sequences (weak scaling, no collective on the data path); the step
+time is the max over ranks and the value counts the bytes of all ranks.
+
+--impl reference times the float64 CPU oracle (the only other implementation of
+the operation) on a bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attention: effective KV-read GB/s vs HBM peak; µs per decode step"
+UNIT = "GB/s"
+FLUSH_BYTES = 512 << 20
+
+DESCRIPTIONS = {
+    "tiny": "tiny paged decode: B2 Hq4 Hkv4 D64 fp16 bs16 ctx {17,40} 8-block pool",
+    "gqa": "GQA decode: B32 Hq32 Hkv8 D128 bf16 bs16 ctx U[512,4096] pool 1.25x shuffled",
+    "long": "long-context GQA decode: B4 Hq32 Hkv8 D128 bf16 bs64 ctx 131072 shuffled",
+    "mla": "MLA absorbed decode: B64 H128 latent 576 (V = first 512) bf16 bs64 ctx U[1024,8192]",
+    "mixed": "mixed continuous-batching decode: B256 Hq64 Hkv8 D128 bf16 bs16 ctx log-U[1,32768]",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="gqa", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed loop runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [l for (t, l) in self.lines if t0 - 0.06 <= t <= t1 + 0.06] or \
+               [l for (_, l) in self.lines]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs"), d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "paged_split_kv_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, kernel_files):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_hash(kernel_files):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def cpu_baseline(w, inp, target_s):
+    """Time the float64 oracle on a bounded sample (leading sequences of the batch)."""
+    import numpy as np
+
+    import oracle
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    nthreads = os.cpu_count() or 1
+    cl = inp["context_lens"]
+    H = w.num_q_heads if w.kind == "gqa" else w.num_heads
+
+    def run(nseq, nheads):
+        pairs = np.array([(b, h) for b in range(nseq) for h in range(nheads)], np.int32)
+        t0 = time.perf_counter()
+        if w.kind == "gqa":
+            oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
+                          inp["block_table"].numpy(), cl.numpy(), inp["scale"], inp["dtype"],
+                          pairs=pairs, nthreads=nthreads)
+        else:
+            oracle.decode_mla(u16(inp["q"]), u16(inp["latent_cache"]), inp["block_table"].numpy(),
+                              cl.numpy(), inp["scale"], inp["dtype"], w.v_dim, pairs=pairs,
+                              nthreads=nthreads)
+        return time.perf_counter() - t0
+
+    # calibrate on the first sequence (all heads), then grow to ~target_s
+    t1 = max(run(1, H), 1e-4)
+    per_tok = t1 / max(int(cl[0]), 1)
+    nseq, acc = 0, 0.0
+    while nseq < w.batch and acc + per_tok * int(cl[nseq]) <= target_s:
+        acc += per_tok * int(cl[nseq])
+        nseq += 1
+    nseq = max(nseq, 1)
+    dt = run(nseq, H)
+    sample_cl = cl[:nseq]
+    nbytes = workloads.kv_bytes(w, sample_cl)
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"first {nseq} of {w.batch} sequences ({int(sample_cl.sum())} tokens, all "
+                      f"{H} heads), float64 C oracle, {dt:.2f} s",
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------ our implementation
+
+def run_ours(args, rank, world, local):
+    import paged_split_kv_attention_b200 as pa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = workloads.get(args.workload)
+    if world > 1:
+        w = workloads.get(args.workload, seed=w.seed + 7919 * rank)
+    inp = workloads.make(w)
+    kv_bytes = workloads.kv_bytes(w, inp["context_lens"])
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    scale = inp["scale"]
+    stream = torch.cuda.current_stream(dev)
+
+    if w.kind == "gqa":
+        desc = pa.gqa_desc(d["q"], d["k_cache"], d["block_table"])
+        out = torch.empty_like(d["q"])
+        call = lambda passes: pa.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"],  # noqa
+                                        d["context_lens"], scale, out=out, workspace=ws,
+                                        passes=passes)
+        kernel_files = ["pa_gqa.cuh", "pa_device.cuh"]
+        kname = "gqa_partition_kernel"
+    else:
+        desc = pa.mla_desc(d["q"], d["latent_cache"], d["block_table"], w.v_dim)
+        out = torch.empty((w.batch, w.num_heads, w.v_dim), dtype=d["q"].dtype, device=dev)
+        call = lambda passes: pa.decode_mla(d["q"], d["latent_cache"], d["block_table"],  # noqa
+                                            d["context_lens"], scale, v_dim=w.v_dim, out=out,
+                                            workspace=ws, passes=passes)
+        kernel_files = ["pa_mla.cuh", "pa_device.cuh"]
+        kname = "mla_partition_kernel"
+    ws = torch.empty(pa.workspace_size(desc), dtype=torch.uint8, device=dev)
+    parts = desc.num_partitions or pa.default_partitions("gqa" if w.kind == "gqa" else "mla",
+                                                         getattr(w, "head_dim", 128))
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=sink)
+
+    for _ in range(args.warmup):
+        flush()
+        call("both")
+    torch.cuda.synchronize()
+    if pa.device_status() != 0:
+        raise RuntimeError("kernel reported an error during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local) if torch.cuda.is_available() else None
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(K):
+        flush()
+        ev[i][0].record(stream)
+        call("partition")
+        ev[i][1].record(stream)
+        call("merge")
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(world)
+    clocks = sampler.stop(t0, t1) if sampler else None
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    part_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    if pa.device_status() != 0:
+        raise RuntimeError("kernel reported an error during the timed loop")
+    local_total = sum(step_ms)
+    total_ms = max_over_ranks(local_total, world, dev)
+    all_bytes = sum_over_ranks(float(kv_bytes), world, dev)
+    ms_per_step = total_ms / K
+    value = all_bytes * K / (total_ms / 1e3) / 1e9
+
+    # e2e: same call through the public API with host buffers, H2D + D2H inside the region
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.pin_memory() for k, v in inp.items() if isinstance(v, torch.Tensor)}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = out_h.numel() * out_h.element_size()
+        Ke = max(3, min(K, 20))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for it in range(2 + Ke):
+            if it == 2:
+                barrier(world)
+                torch.cuda.synchronize()
+                e0.record(stream)
+            for k2, v in host.items():
+                dev_in[k2].copy_(v, non_blocking=True)
+            if w.kind == "gqa":
+                pa.decode(dev_in["q"], dev_in["k_cache"], dev_in["v_cache"], dev_in["block_table"],
+                          dev_in["context_lens"], scale, out=out, workspace=ws)
+            else:
+                pa.decode_mla(dev_in["q"], dev_in["latent_cache"], dev_in["block_table"],
+                              dev_in["context_lens"], scale, v_dim=w.v_dim, out=out, workspace=ws)
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": all_bytes * Ke / (e_ms / 1e3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "includes": "H2D of q, KV pool, block_table, context_lens from pinned host "
+                           "memory + decode + D2H of out, per step"}
+
+    hbm, tf, tf_sus, peak_src = measured_peaks()
+    part_avg_s = statistics.mean(part_ms) / 1e3
+    achieved = kv_bytes / part_avg_s / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(args.workload, kernel_files),
+                "kernel": kname, "peak_source": f"{peak_src} hbm_gbs (copy)",
+                "nominal_frac_8tbs": round(achieved / 8000.0, 4)}
+    if w.kind == "mla":
+        fl = workloads.flops(w, inp["context_lens"])
+        roofline["tensor_tflops"] = round(fl / part_avg_s / 1e12, 1)
+        roofline["tensor_frac"] = round(fl / part_avg_s / 1e12 / tf, 4)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "us_per_step": round(ms_per_step * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": inp["dtype"], "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool)",
+        "config": {"workload": DESCRIPTIONS[args.workload], "batch": w.batch,
+                   "kv_bytes_per_step_per_gpu": kv_bytes,
+                   "tokens_per_step_per_gpu": int(inp["context_lens"].sum()),
+                   "partitions": parts, "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed between steps (512 MiB write + 512 MiB read of another buffer)"},
+        "roofline": roofline, "clocks": clocks, "e2e": e2e,
+        "gpu_launches": 2 * K,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w, inp, args.cpu_seconds)
+        cb.pop("seconds", None)
+        result["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import numpy as np
+
+    import oracle
+    w = workloads.get(args.workload)
+    inp = workloads.make(w)
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    nthreads = os.cpu_count() or 1
+    cl = inp["context_lens"]
+    H = w.num_q_heads if w.kind == "gqa" else w.num_heads
+    # each step: a bounded sample (leading sequences, all heads) sized to ~2 s of CPU work
+    budget_per_step = max(0.5, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+
+    def step(nseq):
+        pairs = np.array([(b, h) for b in range(nseq) for h in range(H)], np.int32)
+        t0 = time.perf_counter()
+        if w.kind == "gqa":
+            oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
+                          inp["block_table"].numpy(), cl.numpy(), inp["scale"], inp["dtype"],
+                          pairs=pairs, nthreads=nthreads)
+        else:
+            oracle.decode_mla(u16(inp["q"]), u16(inp["latent_cache"]), inp["block_table"].numpy(),
+                              cl.numpy(), inp["scale"], inp["dtype"], w.v_dim, pairs=pairs,
+                              nthreads=nthreads)
+        return time.perf_counter() - t0
+
+    t1 = max(step(1), 1e-4)
+    per_tok = t1 / max(int(cl[0]), 1)
+    nseq, acc = 0, 0.0
+    while nseq < w.batch and acc + per_tok * int(cl[nseq]) <= budget_per_step:
+        acc += per_tok * int(cl[nseq])
+        nseq += 1
+    nseq = max(nseq, 1)
+    for _ in range(args.warmup):
+        step(nseq)
+    times = [step(nseq) for _ in range(args.steps)]
+    nbytes = workloads.kv_bytes(w, cl[:nseq])
+    total = sum(times)
+    value = nbytes * len(times) / total / 1e9
+    sample = (f"first {nseq} of {w.batch} sequences ({int(cl[:nseq].sum())} tokens, all {H} "
+              f"heads) per step, float64 C oracle")
+    result = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / len(times) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool)",
+        "config": {"workload": DESCRIPTIONS[args.workload], "batch": w.batch,
+                   "sample_sequences": nseq},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": nthreads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,158 @@
+/*
+ * pa.h -- C ABI of the B200 paged split-KV decode attention library (libpa_b200.so).
+ *
+ * One operation: single-query-token decode attention over a block-paged KV
+ * cache, computed Flash-Decoding style.
+ *
+ *   out[b, h, :] = softmax_t( scale * q[b, h, :] . K_b[t, :] ) V_b[t, :],  t < context_lens[b]
+ *
+ * where logical token t of sequence b lives in row t % block_size of physical
+ * block block_table[b][t / block_size] (page "wenku.it search: paged attention",
+ * vLLM PagedAttention snippet on paged key/value memory).  The KV stream of every
+ * (sequence, kv head) is split along the sequence; each piece is attended
+ * separately, recording the log-sum-exp of each softmax row, and the pieces are
+ * rescaled and reduced at the end (page "cidian.kuaisou.com: flash decoding ++",
+ * snippets on the three Flash-Decoding steps and on loading K/V in parallel then
+ * rescaling and combining).  Query head h reads kv head h / (Hq / Hkv) (grouped
+ * query heads share one kv head, page "bjpcjp.github.io: llms-attention",
+ * MHA -> GQA -> MLA teaser).  The MLA entry points read one shared latent row per
+ * token: the key is the whole kv_dim-wide row and the value its first v_dim dims
+ * (page "wenku.it search: Multi-head Latent Attention (MLA)", DeepSeek-V2
+ * abstract on the compressed latent KV).
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or retains them.  All are dense row-major:
+ *       q            [batch][num_q_heads][head_dim]                 dtype
+ *       k_cache      [num_blocks][num_kv_heads][block_size][head_dim]  dtype
+ *       v_cache      [num_blocks][num_kv_heads][block_size][head_dim]  dtype
+ *       block_table  [batch][max_blocks_per_seq]                    int32
+ *       context_lens [batch]                                        int32
+ *       out          [batch][num_q_heads][head_dim]                 dtype
+ *     MLA: q [batch][num_heads][kv_dim], latent_cache [num_blocks][block_size][kv_dim],
+ *          out [batch][num_heads][v_dim].
+ *     Base addresses must be 16-byte aligned.
+ *   - workspace is caller-owned device scratch of at least the size returned by
+ *     the matching *_workspace_size call; its contents need no initialisation and
+ *     are overwritten by every call.  Two calls in flight at the same time must
+ *     not share a workspace.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is asynchronous on it; nothing is synchronised and no host-side
+ *     copy of device data is made.  context_lens and block_table are read only by
+ *     the GPU.
+ *   - Data contract (checked on the GPU; a violation skips the offending load and
+ *     records an error readable through pa_device_status):
+ *       0 <= context_lens[b] <= max_blocks_per_seq * block_size,
+ *       0 <= block_table[b][j] < num_blocks for j < ceil(context_lens[b] / block_size).
+ *     Entries past ceil(context_lens[b] / block_size) are never read.
+ *     context_lens[b] == 0 gives an all-zero output row.
+ *   - Errors are returned, never thrown; nothing is printed.  Argument errors are
+ *     detected before any launch.  The library keeps no per-call state; it is
+ *     safe to call from several host threads on different streams.
+ */
+#ifndef PA_B200_H
+#define PA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
+  PA_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim, block_size, group size */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, no device) */
+  PA_ERR_BAD_BLOCK_ID = 4,  /* device: block id or context length outside the contract */
+  PA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out */
+  PA_ERR_WORKSPACE = 6      /* workspace null or smaller than required */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Shape of a GQA / MHA / MQA decode call.
+ * Supported: head_dim in {64, 128}; block_size a multiple of 16 up to 1024;
+ * 1 <= num_q_heads / num_kv_heads <= 16; batch >= 0 (0 is a no-op).
+ * num_partitions: number of equal-work pieces the flattened KV stream is cut into
+ * (one CTA each); 0 picks (SM count) x (resident CTAs per SM) for the current device. */
+typedef struct {
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int block_size;
+  int max_blocks_per_seq;
+  int num_blocks;
+  pa_dtype dtype;
+  int num_partitions;
+} pa_desc;
+
+/* Shape of an MLA absorbed decode call.  Supported: num_heads 128, kv_dim 576,
+ * v_dim 512, block_size a multiple of 64 up to 1024, dtype PA_BF16. */
+typedef struct {
+  int batch;
+  int num_heads;
+  int kv_dim;
+  int v_dim;
+  int block_size;
+  int max_blocks_per_seq;
+  int num_blocks;
+  pa_dtype dtype;
+  int num_partitions;
+} pa_mla_desc;
+
+/* Workspace bytes a pa_decode call with this descriptor needs; 0 if the
+ * descriptor is invalid or (num_partitions == 0 and no CUDA device is usable). */
+size_t pa_workspace_size(const pa_desc *desc);
+
+/* Full decode step: partition pass then LSE merge pass, both on `stream`. */
+pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache,
+                    const void *v_cache, const int32_t *block_table,
+                    const int32_t *context_lens, float scale, void *out, void *workspace,
+                    size_t workspace_bytes, void *stream);
+
+/* The two passes of pa_decode, exposed separately so that each can be timed on
+ * its own.  pa_decode_merge must follow pa_decode_partition on the same stream
+ * with the same arguments. */
+pa_status pa_decode_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                              const void *v_cache, const int32_t *block_table,
+                              const int32_t *context_lens, float scale, void *out,
+                              void *workspace, size_t workspace_bytes, void *stream);
+pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *block_table,
+                          const int32_t *context_lens, float scale, void *out,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+size_t pa_mla_workspace_size(const pa_mla_desc *desc);
+
+pa_status pa_decode_mla(const pa_mla_desc *desc, const void *q, const void *latent_cache,
+                        const int32_t *block_table, const int32_t *context_lens, float scale,
+                        void *out, void *workspace, size_t workspace_bytes, void *stream);
+pa_status pa_decode_mla_partition(const pa_mla_desc *desc, const void *q,
+                                  const void *latent_cache, const int32_t *block_table,
+                                  const int32_t *context_lens, float scale, void *out,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+pa_status pa_decode_mla_merge(const pa_mla_desc *desc, const void *q, const void *latent_cache,
+                              const int32_t *block_table, const int32_t *context_lens,
+                              float scale, void *out, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* Number of partitions a call with num_partitions == 0 uses on the current
+ * device (SM count x resident CTAs per SM), or -1 without a usable device.
+ * kind: 0 = GQA with this head_dim, 1 = MLA (head_dim ignored). */
+int pa_default_partitions(int kind, int head_dim);
+
+/* Synchronises `stream`, then returns the first error the kernels recorded on the
+ * current device since the last reset (PA_OK if none); reset != 0 clears it. */
+pa_status pa_device_status(void *stream, int reset);
+
+/* Static description of a status code. */
+const char *pa_status_string(pa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_B200_H */

@@ -1,0 +1,338 @@
+// pa_api.cu -- C ABI of libpa_b200: argument validation, work planning, TMA
+// descriptor set-up and kernel launches.  See include/pa.h for the contract.
+//
+// Everything here runs on the host and is asynchronous with respect to the GPU:
+// no call synchronises, copies device data to the host or allocates memory
+// (pa_device_status is the one documented exception: it synchronises).
+#include "pa.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pa_gqa.cuh"
+#include "pa_merge.cuh"
+#include "pa_mla.cuh"
+
+namespace {
+
+constexpr int kMaxBatch = 4096;            // prefix table lives in shared memory
+constexpr int kMaxPartitions = 1 << 20;
+constexpr float kLog2e = 1.4426950408889634f;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ driver entry
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Row-major [rows][inner] 16-bit tensor, boxes of box_rows x box_inner, 128 B swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t inner, uint64_t rows,
+                 uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+             const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+// Resident CTAs per SM of `kernel` with `smem` dynamic bytes, after raising the
+// kernel's dynamic shared-memory limit (once per device is enough; it is cheap).
+int resident_ctas(const void *kernel, int threads, size_t smem) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return -1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
+    return -1;
+  return n;
+}
+
+// ------------------------------------------------------------------ GQA variants
+
+template <int D, int NT, bool BF16>
+struct GqaVariant {
+  static constexpr int S = D == 128 ? 8 : 16;   // 64 KB ring either way
+  using L = pa::GqaLayout<D, NT, S>;
+  static const void *kernel() {
+    return reinterpret_cast<const void *>(&pa::gqa_partition_kernel<D, NT, BF16, S>);
+  }
+  static void launch(int grid, size_t smem, cudaStream_t st, const CUtensorMap &q,
+                     const CUtensorMap &k, const CUtensorMap &v, const pa::GqaParams &p) {
+    pa::gqa_partition_kernel<D, NT, BF16, S><<<grid, pa::kGqaThreads, smem, st>>>(q, k, v, p);
+  }
+};
+
+template <template <int, int, bool> class F, typename... A>
+bool dispatch_gqa(int D, int NT, bool bf16, A &&...a) {
+#define PA_CASE(d, nt, b)                        \
+  if (D == d && NT == nt && bf16 == b) {         \
+    F<d, nt, b>::run(static_cast<A &&>(a)...);   \
+    return true;                                 \
+  }
+  PA_CASE(128, 1, true) PA_CASE(128, 1, false) PA_CASE(128, 2, true) PA_CASE(128, 2, false)
+  PA_CASE(64, 1, true) PA_CASE(64, 1, false) PA_CASE(64, 2, true) PA_CASE(64, 2, false)
+#undef PA_CASE
+  return false;
+}
+
+template <int D, int NT, bool BF16>
+struct QueryResident {
+  static void run(int B, int *out) {
+    using V = GqaVariant<D, NT, BF16>;
+    *out = resident_ctas(V::kernel(), pa::kGqaThreads, V::L::bytes(B));
+  }
+};
+
+struct GqaPlan {
+  int G = 0, NT = 0, parts = 0;
+  size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
+};
+
+int default_gqa_parts(int D, int NT, bool bf16, int B) {
+  const int sms = sm_count();
+  if (sms <= 0) return -1;
+  int per = -1;
+  if (!dispatch_gqa<QueryResident>(D, NT, bf16, B, &per) || per <= 0) return -1;
+  return sms * per;
+}
+
+pa_status plan_gqa(const pa_desc *d, GqaPlan *pl) {
+  if (!d) return PA_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0 ||
+      d->block_size <= 0 || d->max_blocks_per_seq <= 0 || d->num_blocks <= 0 ||
+      d->num_partitions < 0 || d->num_partitions > kMaxPartitions)
+    return PA_ERR_INVALID_ARG;
+  if (d->dtype != PA_F16 && d->dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (G > 16) return PA_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (d->block_size % pa::kTile || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
+  if (d->batch > kMaxBatch) return PA_ERR_UNSUPPORTED;
+  const int64_t kv_rows = int64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
+  const int64_t q_rows = int64_t(d->batch) * d->num_q_heads;
+  const int64_t cap = int64_t(d->max_blocks_per_seq) * d->block_size;
+  const int64_t max_tiles = int64_t(d->batch) * (cap / pa::kTile) * d->num_kv_heads;
+  if (kv_rows > INT32_MAX || q_rows > INT32_MAX || cap > INT32_MAX || max_tiles > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  pl->G = G;
+  pl->NT = G <= 8 ? 1 : 2;
+  pl->parts = d->num_partitions;
+  if (pl->parts == 0) {
+    pl->parts = default_gqa_parts(d->head_dim, pl->NT, d->dtype == PA_BF16, d->batch);
+    if (pl->parts <= 0) return PA_ERR_CUDA;
+  }
+  const size_t slots = size_t(pl->parts) + size_t(d->batch) * d->num_kv_heads;
+  pl->off_prefix = 0;
+  pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
+  pl->off_o = pl->off_lse + round_up(slots * G * 4, 256);
+  pl->bytes = pl->off_o + slots * G * size_t(d->head_dim) * 4;
+  return PA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status check_gqa_args(const pa_desc *d, const GqaPlan &pl, const void *q, const void *k,
+                         const void *v, const int32_t *bt, const int32_t *cl, const void *out,
+                         const void *ws, size_t ws_bytes) {
+  if (!q || !k || !v || !bt || !cl || !out) return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(bt) & 3u) || (reinterpret_cast<uintptr_t>(cl) & 3u))
+    return PA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < pl.bytes) return PA_ERR_WORKSPACE;
+  (void)d;
+  return PA_OK;
+}
+
+template <int D, int NT, bool BF16>
+struct LaunchPartition {
+  static void run(int grid, cudaStream_t st, const CUtensorMap *maps, const pa::GqaParams *p,
+                  cudaError_t *err) {
+    using V = GqaVariant<D, NT, BF16>;
+    const size_t smem = V::L::bytes(p->B);
+    *err = cudaFuncSetAttribute(V::kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+    if (*err != cudaSuccess) return;
+    V::launch(grid, smem, st, maps[0], maps[1], maps[2], *p);
+    *err = cudaGetLastError();
+  }
+};
+
+template <int DV, bool BF16>
+cudaError_t launch_merge(const pa::MergeParams &mp, cudaStream_t st) {
+  const long long pairs = static_cast<long long>(mp.B) * mp.Hq;
+  const unsigned grid = static_cast<unsigned>((pairs + pa::kMergeWarps - 1) / pa::kMergeWarps);
+  pa::merge_kernel<DV, BF16><<<grid, 32 * pa::kMergeWarps, 0, st>>>(mp);
+  return cudaGetLastError();
+}
+
+cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, cudaStream_t st) {
+  if (DV == 128) return bf16 ? launch_merge<128, true>(mp, st) : launch_merge<128, false>(mp, st);
+  if (DV == 64) return bf16 ? launch_merge<64, true>(mp, st) : launch_merge<64, false>(mp, st);
+  if (DV == 512) return bf16 ? launch_merge<512, true>(mp, st) : launch_merge<512, false>(mp, st);
+  return cudaErrorInvalidValue;
+}
+
+enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
+
+pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, const void *v,
+                  const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
+                  size_t ws_bytes, void *stream) {
+  GqaPlan pl;
+  pa_status s = plan_gqa(d, &pl);
+  if (s != PA_OK) return s;
+  if (d->batch == 0) return PA_OK;
+  s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
+  if (s != PA_OK) return s;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  const bool bf16 = d->dtype == PA_BF16;
+  const int D = d->head_dim;
+
+  if (passes & kPartition) {
+    CUtensorMap maps[3];
+    const uint64_t kv_rows = uint64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
+    if (!make_map_2d(&maps[0], q, bf16, D, uint64_t(d->batch) * d->num_q_heads, 64, 8 * pl.NT) ||
+        !make_map_2d(&maps[1], k, bf16, D, kv_rows, 64, pa::kTile) ||
+        !make_map_2d(&maps[2], v, bf16, D, kv_rows, 64, pa::kTile))
+      return PA_ERR_CUDA;
+    pa::GqaParams p;
+    p.block_table = bt;
+    p.context_lens = cl;
+    p.out = out;
+    p.part_o = reinterpret_cast<float *>(w + pl.off_o);
+    p.part_lse = reinterpret_cast<float *>(w + pl.off_lse);
+    p.prefix_out = reinterpret_cast<int32_t *>(w + pl.off_prefix);
+    p.B = d->batch;
+    p.Hq = d->num_q_heads;
+    p.Hkv = d->num_kv_heads;
+    p.G = pl.G;
+    p.bs = d->block_size;
+    p.mbs = d->max_blocks_per_seq;
+    p.nb = d->num_blocks;
+    p.tiles_per_block = d->block_size / pa::kTile;
+    p.parts = pl.parts;
+    p.scale_log2 = scale * kLog2e;
+    cudaError_t err = cudaSuccess;
+    if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, pl.parts, st, maps, &p, &err))
+      return PA_ERR_UNSUPPORTED;
+    if (err != cudaSuccess) return PA_ERR_CUDA;
+  }
+  if (passes & kMerge) {
+    pa::MergeParams mp;
+    mp.part_o = reinterpret_cast<const float *>(w + pl.off_o);
+    mp.part_lse = reinterpret_cast<const float *>(w + pl.off_lse);
+    mp.prefix = reinterpret_cast<const int32_t *>(w + pl.off_prefix);
+    mp.out = out;
+    mp.B = d->batch;
+    mp.Hq = d->num_q_heads;
+    mp.Hkv = d->num_kv_heads;
+    mp.G = pl.G;
+    mp.parts = pl.parts;
+    if (merge_dispatch(D, bf16, mp, st) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+size_t pa_workspace_size(const pa_desc *desc) {
+  GqaPlan pl;
+  if (plan_gqa(desc, &pl) != PA_OK) return 0;
+  return pl.bytes;
+}
+
+pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_table, const int32_t *context_lens, float scale,
+                    void *out, void *workspace, size_t workspace_bytes, void *stream) {
+  return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                              const void *v_cache, const int32_t *block_table,
+                              const int32_t *context_lens, float scale, void *out,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+  return run_gqa(kPartition, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *block_table,
+                          const int32_t *context_lens, float scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+  return run_gqa(kMerge, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream);
+}
+
+int pa_default_partitions(int kind, int head_dim) {
+  if (kind == 0) {
+    if (head_dim != 64 && head_dim != 128) return -1;
+    return default_gqa_parts(head_dim, 1, true, 256);
+  }
+  return pa_mla_default_parts();
+}
+
+pa_status pa_device_status(void *stream, int reset) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_status, sizeof(int)) != cudaSuccess) return PA_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(pa::g_status, &zero, sizeof(int)) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return static_cast<pa_status>(v);
+}
+
+const char *pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_BAD_BLOCK_ID: return "block id or context length outside the data contract";
+    case PA_ERR_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

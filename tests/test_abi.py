@@ -1,0 +1,99 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every entry
+point include/pa.h declares, and rejects bad arguments on the host before any
+CUDA call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_split_kv_attention_b200 import _build
+    _build.build()
+    import paged_split_kv_attention_b200 as pa
+    return pa.library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(pa_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("pa_decode", "pa_decode_mla", "pa_workspace_size", "pa_mla_workspace_size",
+                 "pa_decode_partition", "pa_decode_merge", "pa_device_status",
+                 "pa_status_string"):
+        assert want in names, names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in pa.h but not exported"
+
+
+def test_status_strings(lib):
+    import paged_split_kv_attention_b200 as pa
+    for s in range(7):
+        assert pa.status_string(s)
+    assert "unknown" in pa.status_string(99)
+
+
+def _desc(**kw):
+    import paged_split_kv_attention_b200 as pa
+    d = dict(batch=4, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+             max_blocks_per_seq=64, num_blocks=300, dtype=pa.PA_BF16, num_partitions=10)
+    d.update(kw)
+    return pa.PADesc(**d)
+
+
+def test_workspace_size_is_host_computable(lib):
+    import paged_split_kv_attention_b200 as pa
+    n = lib.pa_workspace_size(ctypes.byref(_desc()))
+    slots = 10 + 4 * 8
+    assert n >= slots * 4 * 128 * 4 + slots * 4 * 4 + 5 * 4
+    assert lib.pa_workspace_size(ctypes.byref(_desc(num_partitions=20))) > n
+    assert lib.pa_workspace_size(None) == 0
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(num_q_heads=30), 1),          # Hq not a multiple of Hkv
+    (dict(head_dim=96), 2),             # unsupported head dim
+    (dict(block_size=8), 2),            # block size not a multiple of 16
+    (dict(num_q_heads=8 * 17), 2),      # group of 17 heads
+    (dict(batch=-1), 1),
+    (dict(num_partitions=-3), 1),
+    (dict(dtype=7), 1),
+])
+def test_invalid_descriptors_are_rejected_before_launch(lib, bad, status):
+    d = _desc(**bad)
+    z = ctypes.c_void_p(0x1000)
+    rc = lib.pa_decode(ctypes.byref(d), z, z, z, z, z, 0.1, z, z, 1 << 30, None)
+    assert rc == status
+    assert lib.pa_workspace_size(ctypes.byref(d)) == 0
+
+
+def test_null_pointers_and_small_workspace_are_rejected(lib):
+    import paged_split_kv_attention_b200 as pa
+    d = _desc()
+    z = ctypes.c_void_p(0x1000)
+    null = ctypes.c_void_p(0)
+    assert lib.pa_decode(ctypes.byref(d), null, z, z, z, z, 0.1, z, z, 1 << 30, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_decode(ctypes.byref(d), z, z, z, z, z, 0.1, z, z, 16, None) == pa.PA_ERR_WORKSPACE
+    assert lib.pa_decode(ctypes.byref(d), ctypes.c_void_p(0x1002), z, z, z, z, 0.1, z, z, 1 << 30,
+                         None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_decode(ctypes.byref(d), z, z, z, z, z, float("nan"), z, z, 1 << 30,
+                         None) == pa.PA_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(lib):
+    d = _desc(batch=0)
+    null = ctypes.c_void_p(0)
+    assert lib.pa_decode(ctypes.byref(d), null, null, null, null, null, 0.1, null, null, 0, None) == 0
