@@ -14,7 +14,6 @@
 #include <mutex>
 
 #include "pa_gqa.cuh"
-#include "pa_merge.cuh"
 #include "pa_mla.cuh"
 
 namespace {
@@ -84,14 +83,14 @@ int resident_ctas(const void *kernel, int threads, size_t smem) {
 
 template <int D, int NT, bool BF16>
 struct GqaVariant {
-  static constexpr int S = D == 128 ? 8 : 16;   // 64 KB ring either way
-  using L = pa::GqaLayout<D, NT, S>;
+  static constexpr int R = D == 128 ? 3 : 6;    // 24 KB ring per warp either way
+  using L = pa::GqaLayout<D, NT, R>;
   static const void *kernel() {
-    return reinterpret_cast<const void *>(&pa::gqa_partition_kernel<D, NT, BF16, S>);
+    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R>);
   }
-  static void launch(int grid, size_t smem, cudaStream_t st, const CUtensorMap &q,
-                     const CUtensorMap &k, const CUtensorMap &v, const pa::GqaParams &p) {
-    pa::gqa_partition_kernel<D, NT, BF16, S><<<grid, pa::kGqaThreads, smem, st>>>(q, k, v, p);
+  static void launch(int grid, size_t smem, cudaStream_t st, const CUtensorMap &k,
+                     const CUtensorMap &v, const pa::GqaParams &p) {
+    pa::gqa_decode_kernel<D, NT, BF16, R><<<grid, pa::kGqaThreads, smem, st>>>(k, v, p);
   }
 };
 
@@ -118,7 +117,7 @@ struct QueryResident {
 
 struct GqaPlan {
   int G = 0, NT = 0, parts = 0;
-  size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
+  size_t off_cnt = 0, cnt_bytes = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
 int default_gqa_parts(int D, int NT, bool bf16, int B) {
@@ -155,9 +154,11 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl) {
     pl->parts = default_gqa_parts(d->head_dim, pl->NT, d->dtype == PA_BF16, d->batch);
     if (pl->parts <= 0) return PA_ERR_CUDA;
   }
-  const size_t slots = size_t(pl->parts) + size_t(d->batch) * d->num_kv_heads;
-  pl->off_prefix = 0;
-  pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
+  // one partial slot per (warp piece, segment) pair a piece can end: piece + segment
+  const size_t slots = size_t(pl->parts) * pa::kWarps + size_t(d->batch) * d->num_kv_heads;
+  pl->off_cnt = 0;
+  pl->cnt_bytes = size_t(d->batch) * d->num_kv_heads * 4;
+  pl->off_lse = round_up(pl->cnt_bytes, 256);
   pl->off_o = pl->off_lse + round_up(slots * G * 4, 256);
   pl->bytes = pl->off_o + slots * G * size_t(d->head_dim) * 4;
   return PA_OK;
@@ -186,27 +187,12 @@ struct LaunchPartition {
     *err = cudaFuncSetAttribute(V::kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(smem));
     if (*err != cudaSuccess) return;
-    V::launch(grid, smem, st, maps[0], maps[1], maps[2], *p);
+    V::launch(grid, smem, st, maps[0], maps[1], *p);
     *err = cudaGetLastError();
   }
 };
 
-template <int DV, bool BF16>
-cudaError_t launch_merge(const pa::MergeParams &mp, cudaStream_t st) {
-  const long long pairs = static_cast<long long>(mp.B) * mp.Hq;
-  const unsigned grid = static_cast<unsigned>((pairs + pa::kMergeWarps - 1) / pa::kMergeWarps);
-  pa::merge_kernel<DV, BF16><<<grid, 32 * pa::kMergeWarps, 0, st>>>(mp);
-  return cudaGetLastError();
-}
-
-cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, cudaStream_t st) {
-  if (DV == 128) return bf16 ? launch_merge<128, true>(mp, st) : launch_merge<128, false>(mp, st);
-  if (DV == 64) return bf16 ? launch_merge<64, true>(mp, st) : launch_merge<64, false>(mp, st);
-  if (DV == 512) return bf16 ? launch_merge<512, true>(mp, st) : launch_merge<512, false>(mp, st);
-  return cudaErrorInvalidValue;
-}
-
-enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
+enum Pass { kPrepare = 1, kLaunch = 2, kBoth = 3 };
 
 pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, const void *v,
                   const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
@@ -215,28 +201,36 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
   pa_status s = plan_gqa(d, &pl);
   if (s != PA_OK) return s;
   if (d->batch == 0) return PA_OK;
-  s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
-  if (s != PA_OK) return s;
-  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (passes == kPrepare) {
+    if (!ws || !aligned16(ws) || ws_bytes < pl.bytes) return PA_ERR_WORKSPACE;
+  } else {
+    s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
+    if (s != PA_OK) return s;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
   const bool bf16 = d->dtype == PA_BF16;
   const int D = d->head_dim;
 
-  if (passes & kPartition) {
-    CUtensorMap maps[3];
+  if (passes & kPrepare) {
+    // per-segment piece counters of the fused merge start from zero
+    if (cudaMemsetAsync(w + pl.off_cnt, 0, pl.cnt_bytes, st) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  if (passes & kLaunch) {
+    CUtensorMap maps[2];
     const uint64_t kv_rows = uint64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
-    if (!make_map_2d(&maps[0], q, bf16, D, uint64_t(d->batch) * d->num_q_heads, 64, 8 * pl.NT) ||
-        !make_map_2d(&maps[1], k, bf16, D, kv_rows, 64, pa::kTile) ||
-        !make_map_2d(&maps[2], v, bf16, D, kv_rows, 64, pa::kTile))
+    if (!make_map_2d(&maps[0], k, bf16, D, kv_rows, 64, pa::kTile) ||
+        !make_map_2d(&maps[1], v, bf16, D, kv_rows, 64, pa::kTile))
       return PA_ERR_CUDA;
     pa::GqaParams p;
+    p.q = static_cast<const uint16_t *>(q);
     p.block_table = bt;
     p.context_lens = cl;
     p.out = out;
     p.part_o = reinterpret_cast<float *>(w + pl.off_o);
     p.part_lse = reinterpret_cast<float *>(w + pl.off_lse);
-    p.prefix_out = reinterpret_cast<int32_t *>(w + pl.off_prefix);
+    p.seg_count = reinterpret_cast<int32_t *>(w + pl.off_cnt);
     p.B = d->batch;
     p.Hq = d->num_q_heads;
     p.Hkv = d->num_kv_heads;
@@ -251,19 +245,6 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
     if (err != cudaSuccess) return PA_ERR_CUDA;
-  }
-  if (passes & kMerge) {
-    pa::MergeParams mp;
-    mp.part_o = reinterpret_cast<const float *>(w + pl.off_o);
-    mp.part_lse = reinterpret_cast<const float *>(w + pl.off_lse);
-    mp.prefix = reinterpret_cast<const int32_t *>(w + pl.off_prefix);
-    mp.out = out;
-    mp.B = d->batch;
-    mp.Hq = d->num_q_heads;
-    mp.Hkv = d->num_kv_heads;
-    mp.G = pl.G;
-    mp.parts = pl.parts;
-    if (merge_dispatch(D, bf16, mp, st) != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
 }
@@ -287,19 +268,17 @@ pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache, con
                  workspace, workspace_bytes, stream);
 }
 
-pa_status pa_decode_partition(const pa_desc *desc, const void *q, const void *k_cache,
-                              const void *v_cache, const int32_t *block_table,
-                              const int32_t *context_lens, float scale, void *out,
-                              void *workspace, size_t workspace_bytes, void *stream) {
-  return run_gqa(kPartition, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+pa_status pa_decode_prepare(const pa_desc *desc, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kPrepare, desc, nullptr, nullptr, nullptr, nullptr, nullptr, 1.f, nullptr,
                  workspace, workspace_bytes, stream);
 }
 
-pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cache,
-                          const void *v_cache, const int32_t *block_table,
-                          const int32_t *context_lens, float scale, void *out, void *workspace,
-                          size_t workspace_bytes, void *stream) {
-  return run_gqa(kMerge, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+pa_status pa_decode_launch(const pa_desc *desc, const void *q, const void *k_cache,
+                           const void *v_cache, const int32_t *block_table,
+                           const int32_t *context_lens, float scale, void *out, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+  return run_gqa(kLaunch, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
                  workspace, workspace_bytes, stream);
 }
 

@@ -1,72 +1,79 @@
-// pa_gqa.cuh -- partition pass of paged split-KV decode for grouped query heads.
+// pa_gqa.cuh -- paged split-KV decode for grouped query heads (GQA / MHA / MQA):
+// partition pass and LSE merge in one kernel.
 //
 // What it computes (page "cidian.kuaisou.com: flash decoding ++", snippets on the
 // three Flash-Decoding steps): the KV stream of every (sequence, kv head) is cut
 // into pieces along the sequence; for each piece and each of the G query heads
 // that share the kv head, attention over the piece's tokens is computed with a
 // running max and sum, and the piece's normalised output plus the log-sum-exp of
-// its softmax row are recorded for the merge pass.  A piece that covers a whole
+// its softmax row are recorded; the pieces are then rescaled by their
+// log-sum-exps and reduced into the output.  A piece that covers a whole
 // (sequence, kv head) writes the final output directly.
 //
 // How the pieces are chosen.  The KV stream is flattened into 16-token tiles in
-// (sequence, kv head, tile) order; grid CTA c owns tiles [c*T/P, (c+1)*T/P) of the
-// T tiles, so every CTA reads the same number of bytes whatever the mix of
-// context lengths.  Where a CTA's range crosses (sequence, kv head) boundaries it
-// produces one partial result per segment it touches (slot c + segment).  The
-// split points therefore fall where the work balances, not at a fixed length.
+// (sequence, kv head, tile) order and cut into P equal runs of tiles, one per
+// warp of a persistent grid (P = CTAs x 8 warps): every warp reads the same
+// number of bytes whatever the mix of context lengths.  Where a warp's run
+// crosses (sequence, kv head) boundaries -- a "segment" -- it produces one
+// result per segment it touches.  The split points therefore fall where the
+// work balances, not at a fixed length.
+//
+// Merge.  A warp that ends a segment it shares with other warps writes its
+// normalised partial and log-sum-exp (slot = warp piece + segment), bumps the
+// segment's counter and, if it is the last of the segment's pieces to finish,
+// merges all of them (they are still in L2) into the output.  Other warps keep
+// streaming meanwhile; no CTA-wide barrier exists after the prologue.
 //
 // Data movement (the pages ask that K and V be loaded in parallel as fast as
-// possible, then rescaled and combined).  Warp 0 is a producer: it walks the
-// CTA's tiles, looks up each tile's physical block through the block table and
-// issues TMA tensor copies of the 16 x D K and V tiles (128-byte swizzle, L2
-// evict-first) into an S-stage shared-memory ring guarded by mbarriers.  Warps
-// 1..4 consume tiles round-robin.  Per tile a consumer computes S^T = K Q^T with
+// possible, then rescaled and combined).  Each warp is its own pipeline: lane 0
+// issues TMA tensor copies (128-byte swizzle, L2 evict-first) of the next R
+// tiles' K and V (16 x D each, physical block looked up through the block table
+// by a 32-tile look-ahead held one tile per lane) into the warp's R-stage ring,
+// each stage guarded by an mbarrier.  Per tile the warp computes S^T = K Q^T with
 // mma.sync m16n8k16 (tokens on M, the group's heads on N), the online softmax in
-// registers (max over tokens with three xor shuffles, sums kept per lane), and
+// registers (max over tokens with three xor shuffles, sums kept per lane) and
 // O^T += V^T P with V^T fragments from ldmatrix.trans and P moved to the B
-// operand layout with movmatrix (as a 16-bit hi + lo pair, two MMAs).  At the end of each segment the four consumer
-// warps combine their (max, sum, O) states through shared memory.
+// operand layout with movmatrix (as a 16-bit hi + lo pair, two MMAs).  The query
+// fragments of the next segment are prefetched into registers.
 #pragma once
 
 #include "pa_device.cuh"
 
 namespace pa {
 
-constexpr int kTile = 16;            // tokens per pipeline tile
-constexpr int kConsumerWarps = 4;
-constexpr int kGqaThreads = 32 * (1 + kConsumerWarps);
+constexpr int kTile = 16;               // tokens per pipeline tile
+constexpr int kWarps = 8;               // independent streaming warps per CTA
+constexpr int kGqaThreads = 32 * kWarps;
+constexpr int kMergeFloats = 256;       // per-warp staging for the merge weights
 
 struct GqaParams {
+  const uint16_t *q;            // [B][Hq][D]
   const int32_t *block_table;   // [B][mbs]
   const int32_t *context_lens;  // [B]
   void *out;                    // [B][Hq][D] 16-bit
   float *part_o;                // [slots][G][D]
-  float *part_lse;              // [slots][G], log2 domain
-  int32_t *prefix_out;          // [B+1] tiles per kv head, written by CTA 0 for the merge
+  float *part_lse;              // [slots][G], log2 units
+  int32_t *seg_count;           // [B*Hkv] finished pieces per segment, zero at launch
   int B, Hq, Hkv, G, bs, mbs, nb;
   int tiles_per_block;          // bs / 16
   int parts;                    // gridDim.x
   float scale_log2;             // scale * log2(e)
 };
 
-template <int D, int NT, int S>
+template <int D, int NT, int R>
 struct GqaLayout {
   static constexpr int kHeads = 8 * NT;            // group width padded to the MMA N
   static constexpr int kKTile = kTile * D * 2;     // bytes of one K (or V) tile
   static constexpr int kStage = 2 * kKTile;
-  static constexpr int kQTile = kHeads * D * 2;
-  static constexpr int kCombStride = D + 4;        // floats per head row (bank spread)
-  static constexpr int kCombWarp = kHeads * kCombStride * 4 + 2 * kHeads * 4;
-  static constexpr int ring = 0;
-  static constexpr int qbuf = ring + S * kStage;
-  static constexpr int comb = qbuf + 2 * kQTile;
-  static constexpr int bars = comb + kConsumerWarps * kCombWarp;
-  static constexpr int nbars = 2 * S + 4;
-  static constexpr int info = bars + nbars * 8;     // int stage_ntok[S]
-  static constexpr int flags = info + S * 4;        // abort flag + scan scratch (16 ints)
+  static constexpr int ring = 0;                   // warp w: stages [w*R, (w+1)*R)
+  static constexpr int merge = ring + kWarps * R * kStage;
+  static constexpr int bars = merge + kWarps * kMergeFloats * 4;
+  static constexpr int nbars = kWarps * R;
+  static constexpr int info = bars + nbars * 8;     // int stage_valid[kWarps * R]
+  static constexpr int flags = info + nbars * 4;    // abort flag + scan scratch
   static constexpr int prefix = flags + 64;         // int prefix[B + 1]
   static size_t bytes(int B) { return 1024 + prefix + static_cast<size_t>(B + 1) * 4; }
-  static_assert(kStage % 1024 == 0 && kQTile % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kStage % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(bars % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
@@ -119,23 +126,123 @@ __device__ __forceinline__ void locate_tile(const int *prefix, int B, int Hkv, l
   j = static_cast<int>(r - static_cast<long long>(kvh) * P);
 }
 
-template <int D, int NT, bool BF16, int S>
+// Cache row of the first token of flattened tile t, or -1 if its block id is
+// outside [0, nb) (recorded, never dereferenced).
+__device__ __forceinline__ int tile_row(const GqaParams &p, const int *prefix, long long t) {
+  int b, kvh, j;
+  locate_tile(prefix, p.B, p.Hkv, t, b, kvh, j);
+  const int jb = j / p.tiles_per_block;
+  const int blk = __ldg(&p.block_table[static_cast<long long>(b) * p.mbs + jb]);
+  if (blk < 0 || blk >= p.nb) return -1;
+  return (blk * p.Hkv + kvh) * p.bs + (j - jb * p.tiles_per_block) * kTile;
+}
+
+// Query B-operand fragments (Q^T: d x heads) of group (b, kvh): for n-tile nt and
+// k-step ks, lane holds Q[head 8nt+g][16ks+2tq .. +1] and Q[..][16ks+8+2tq .. +1];
+// heads past the group are zero.
+template <int D, int NT>
+__device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int lane,
+                                       uint32_t (&qf)[NT][D / 16][2]) {
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int h = nt * 8 + g;
+    const bool ok = h < p.G;
+    const uint32_t *row = reinterpret_cast<const uint32_t *>(
+        p.q + (static_cast<long long>(b) * p.Hq + kvh * p.G + (ok ? h : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qf[nt][ks][0] = ok ? __ldg(row + ks * 8 + tq) : 0u;
+      qf[nt][ks][1] = ok ? __ldg(row + ks * 8 + 4 + tq) : 0u;
+    }
+  }
+}
+
+// Third Flash-Decoding step for one split segment, run by the warp that finished
+// the segment last: pieces pc in [g0, g1] left normalised partials o_pc and
+// log-sum-exps lse_pc (log2 units) in slot pc + seg;
+//   out = sum 2^(lse - M) o / sum 2^(lse - M),  M = max lse,
+// with M tracked online over chunks of pieces staged in shared memory.
+template <int D, bool BF16>
+__device__ __noinline__ void warp_merge(const float *part_o, const float *part_lse,
+                                        uint16_t *out_rows, int G, int pieces_total,
+                                        long long seg, int g0, int g1, long long TP,
+                                        float *stage, int lane) {
+  constexpr int F4 = D / 4;                         // float4 per head row
+  const int items = (G * F4 + 31) / 32;              // float4 items per lane
+  const int chunk = kMergeFloats / G;
+  float Mrun[16], Wrun[16];
+  float4 acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    Mrun[i] = -INFINITY;
+    Wrun[i] = 0.f;
+    acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int cs = g0; cs <= g1; cs += chunk) {
+    const int ce = min(g1, cs + chunk - 1);
+    const int n = (ce - cs + 1) * G;
+    for (int i = lane; i < n; i += 32) {
+      const int pc = cs + i / G, h = i - (i / G) * G;
+      stage[i] = piece_begin(pc + 1, TP, pieces_total) > piece_begin(pc, TP, pieces_total)
+                     ? __ldcg(&part_lse[(pc + seg) * G + h])
+                     : -INFINITY;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i >= items) break;
+      const int f = lane + 32 * i;
+      if (f >= G * F4) continue;
+      const int h = f / F4;
+      float Mc = -INFINITY;
+      for (int pc = cs; pc <= ce; ++pc) Mc = fmaxf(Mc, stage[(pc - cs) * G + h]);
+      const float Mn = fmaxf(Mrun[i], Mc);
+      if (Mn == -INFINITY) continue;
+      const float r = Mrun[i] == -INFINITY ? 0.f : exp2f(Mrun[i] - Mn);
+      acc[i].x *= r; acc[i].y *= r; acc[i].z *= r; acc[i].w *= r;
+      Wrun[i] *= r;
+      Mrun[i] = Mn;
+    }
+    for (int pc = cs; pc <= ce; ++pc) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i >= items) break;
+        const int f = lane + 32 * i;
+        if (f >= G * F4) continue;
+        const int h = f / F4;
+        const float lse = stage[(pc - cs) * G + h];
+        if (lse == -INFINITY) continue;
+        const float w = exp2f(lse - Mrun[i]);
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(part_o + ((pc + seg) * G) * D) + f);
+        Wrun[i] += w;
+        acc[i].x += w * v.x; acc[i].y += w * v.y; acc[i].z += w * v.z; acc[i].w += w * v.w;
+      }
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i >= items) break;
+    const int f = lane + 32 * i;
+    if (f >= G * F4) continue;
+    const float inv = Wrun[i] > 0.f ? 1.f / Wrun[i] : 0.f;
+    const uint32_t lo = pack2<BF16>(acc[i].x * inv, acc[i].y * inv);
+    const uint32_t hi = pack2<BF16>(acc[i].z * inv, acc[i].w * inv);
+    *reinterpret_cast<uint2 *>(out_rows + static_cast<long long>(f) * 4) = make_uint2(lo, hi);
+  }
+}
+
+template <int D, int NT, bool BF16, int R>
 __global__ void __launch_bounds__(kGqaThreads, 1)
-gqa_partition_kernel(const __grid_constant__ CUtensorMap tm_q,
-                     const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
-  using L = GqaLayout<D, NT, S>;
-  static_assert(S % kConsumerWarps == 0, "each consumer warp owns fixed ring stages");
+gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
+  using L = GqaLayout<D, NT, R>;
   constexpr int KS = D / 16;                 // k-steps of the score MMA / m-tiles of the PV MMA
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::bars);
-  uint64_t *empty = full + S;
-  uint64_t *qfull = empty + S;
-  uint64_t *qempty = qfull + 2;
-  int *stage_ntok = reinterpret_cast<int *>(sm + L::info);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::flags);
   int *scan_scratch = reinterpret_cast<int *>(sm + L::flags) + 4;
   int *prefix = reinterpret_cast<int *>(sm + L::prefix);
@@ -144,162 +251,114 @@ gqa_partition_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int c = blockIdx.x;
   const int cap = p.mbs * p.bs;
 
+  // Warm L2 with this CTA's share of the block table while the lengths load.
+  {
+    const char *tb = reinterpret_cast<const char *>(p.block_table);
+    const long long bytes = static_cast<long long>(p.B) * p.mbs * 4;
+    const long long lo = bytes * c / p.parts, hi = bytes * (c + 1) / p.parts;
+    for (long long off = (lo & ~127ll) + tid * 128ll; off < hi; off += kGqaThreads * 128ll)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + off));
+  }
   tiles_prefix<kGqaThreads>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0);
-  if (c == 0)
-    for (int i = tid; i <= p.B; i += kGqaThreads) p.prefix_out[i] = prefix[i];
+  // sequences with no tokens get an all-zero output row (spread over the grid)
+  for (int b = c; b < p.B; b += p.parts)
+    if (prefix[b + 1] == prefix[b])
+      for (int i = tid; i < p.Hq * D; i += kGqaThreads)
+        reinterpret_cast<uint16_t *>(p.out)[static_cast<long long>(b) * p.Hq * D + i] = 0;
 
   const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
-  const long long t_begin = piece_begin(c, TP, p.parts);
-  const long long t_end = piece_begin(c + 1, TP, p.parts);
-  if (t_begin >= t_end) return;
+  const int pieces = p.parts * kWarps;
+  const int gw = c * kWarps + warp;                     // this warp's piece
+  const long long wb = piece_begin(gw, TP, pieces);
+  const long long we = piece_begin(gw + 1, TP, pieces);
 
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&qfull[s], 1);
-      mbar_init(&qempty[s], kConsumerWarps);
-    }
-    *abort_flag = 0;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::bars) + warp * R;
+  int *stage_valid = reinterpret_cast<int *>(sm + L::info) + warp * R;
+  uint8_t *ring = sm + L::ring + warp * R * L::kStage;
+  float *mstage = reinterpret_cast<float *>(sm + L::merge) + warp * kMergeFloats;
+  if (lane == 0) {
+    for (int s = 0; s < R; ++s) mbar_init(&full[s], 1);
+    if (warp == 0) *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  if (wb >= we) return;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-    }
-    const uint64_t policy = l2_evict_first_policy();
-    long long issued = 0;     // tiles issued (lane 0)
-    int q_issued = 0;         // query tiles issued (lane 0)
-    int seg_k = -1;           // segment ordinal in this CTA (lane 0)
-    bool aborted = false;
-    for (long long base = t_begin; base < t_end && !aborted; base += 32) {
-      const long long t = base + lane;
-      int b = 0, kvh = 0, j = 0, ntok = 0, row = 0, seg_start = 0;
-      if (t < t_end) {
-        locate_tile(prefix, p.B, p.Hkv, t, b, kvh, j);
-        const int ctx = clamp_ctx(p.context_lens[b], cap);
-        ntok = min(kTile, ctx - j * kTile);
-        const int jb = j / p.tiles_per_block;
-        const int blk = p.block_table[static_cast<long long>(b) * p.mbs + jb];
-        if (blk < 0 || blk >= p.nb) {
-          record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
-          ntok = 0;
-        } else {
-          row = (blk * p.Hkv + kvh) * p.bs + (j - jb * p.tiles_per_block) * kTile;
-        }
-        seg_start = (j == 0 || t == t_begin) ? 1 : 0;
-      }
-      const int n = static_cast<int>(min(32ll, t_end - base));
-      for (int i = 0; i < n; ++i) {
-        const int bi = __shfl_sync(0xffffffffu, b, i);
-        const int kvi = __shfl_sync(0xffffffffu, kvh, i);
-        const int ni = __shfl_sync(0xffffffffu, ntok, i);
-        const int ri = __shfl_sync(0xffffffffu, row, i);
-        const int si = __shfl_sync(0xffffffffu, seg_start, i);
-        if (lane == 0 && !aborted) {
-          if (si) {
-            ++seg_k;
-            const int qs = seg_k & 1;
-            if (!mbar_wait(&qempty[qs], ((seg_k >> 1) & 1) ^ 1, abort_flag)) {
-              aborted = true;
-            } else {
-              mbar_arrive_expect_tx(&qfull[qs], L::kQTile);
-              uint8_t *qdst = sm + L::qbuf + qs * L::kQTile;
-#pragma unroll
-              for (int x = 0; x < D; x += 64)
-                tma_load_2d(qdst + (x / 64) * L::kHeads * 128, &tm_q, &qfull[qs], x,
-                            bi * p.Hq + kvi * p.G);
-              q_issued = seg_k + 1;
-            }
-          }
-          const long long li = base + i - t_begin;
-          const int st = static_cast<int>(li % S);
-          const uint32_t ph = static_cast<uint32_t>((li / S) & 1);
-          if (!aborted && !mbar_wait(&empty[st], ph ^ 1, abort_flag)) aborted = true;
-          if (!aborted) {
-            stage_ntok[st] = ni;
-            if (ni > 0) {
-              mbar_arrive_expect_tx(&full[st], L::kStage);
-              uint8_t *kdst = sm + L::ring + st * L::kStage;
-#pragma unroll
-              for (int x = 0; x < D; x += 64) {
-                tma_load_2d_hint(kdst + (x / 64) * kTile * 128, &tm_k, &full[st], x, ri, policy);
-                tma_load_2d_hint(kdst + L::kKTile + (x / 64) * kTile * 128, &tm_v, &full[st], x,
-                                 ri, policy);
-              }
-            } else {
-              mbar_arrive(&full[st]);
-            }
-            issued = li + 1;
-          }
-        }
-      }
-      aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
-    }
-    if (lane == 0 && aborted) {
-      // Leave no copy in flight into this CTA's shared memory: wait (bounded) for
-      // the most recent S tiles and the last two Q tiles to land.
-      volatile int never = 0;
-      for (long long li = issued > S ? issued - S : 0; li < issued; ++li)
-        mbar_wait(&full[li % S], static_cast<uint32_t>((li / S) & 1), &never);
-      for (int k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k)
-        mbar_wait(&qfull[k & 1], static_cast<uint32_t>((k >> 1) & 1), &never);
-    }
-    return;
+  const uint64_t policy = l2_evict_first_policy();
+  if (lane == 0) {
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
   }
 
-  // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;
+  // ---- look-ahead: lane i holds the cache row of tile la_base + i
+  long long la_base = wb;
+  int la_row = (wb + lane < we) ? tile_row(p, prefix, wb + lane) : 0;
+  long long nx_base = wb + 32;
+  int nx_row = (nx_base + lane < we) ? tile_row(p, prefix, nx_base + lane) : 0;
+  long long issued = wb;                              // next tile to issue
+
+  // Issue tile `issued` into its stage (lane 0 does the copy; all lanes call).
+  auto issue_next = [&]() {
+    if (issued >= we) return;
+    if (issued >= la_base + 32) {                     // slide the look-ahead window
+      la_base = nx_base;
+      la_row = nx_row;
+      nx_base += 32;
+      nx_row = (nx_base + lane < we) ? tile_row(p, prefix, nx_base + lane) : 0;
+    }
+    const int row = __shfl_sync(0xffffffffu, la_row, static_cast<int>(issued - la_base));
+    const long long n = issued - wb;
+    const int st = static_cast<int>(n % R);
+    if (lane == 0) {
+      if (row < 0) {
+        record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
+        stage_valid[st] = 0;
+        mbar_arrive(&full[st]);
+      } else {
+        stage_valid[st] = 1;
+        mbar_arrive_expect_tx(&full[st], L::kStage);
+        uint8_t *dst = ring + st * L::kStage;
+#pragma unroll
+        for (int x = 0; x < D; x += 64) {
+          tma_load_2d_hint(dst + (x / 64) * kTile * 128, &tm_k, &full[st], x, row, policy);
+          tma_load_2d_hint(dst + L::kKTile + (x / 64) * kTile * 128, &tm_v, &full[st], x, row,
+                           policy);
+        }
+      }
+    }
+    ++issued;
+  };
+  for (int s = 0; s < R; ++s) issue_next();
+
   const int g = lane >> 2;          // fragment row group
   const int tq = lane & 3;          // thread in quad
-  float *comb_all = reinterpret_cast<float *>(sm + L::comb);
-  float *comb_me = comb_all + cw * (L::kCombWarp / 4);
-  const uint32_t ring_base = smem_u32(sm + L::ring);
-  const uint32_t q_base = smem_u32(sm + L::qbuf);
-  // per-lane ldmatrix row/column offsets (see fragment layouts in the header comment)
+  const uint32_t ring_base = smem_u32(ring);
+  // per-lane ldmatrix row/column offsets (see the fragment layouts above)
   const int k_row = (lane & 7) + ((lane >> 3) & 1) * 8, k_col = (lane >> 4) * 8;
   const int v_row = (lane & 7) + (lane >> 4) * 8, v_col = ((lane >> 3) & 1) * 8;
-  const int q_row = lane & 7, q_col = (lane >> 3) * 8;
 
-  long long t = t_begin;
-  int seg_k = -1;
-  while (t < t_end) {
-    ++seg_k;
-    int b, kvh, j0;
-    locate_tile(prefix, p.B, p.Hkv, t, b, kvh, j0);
+  // current and next segment
+  int b, kvh, j0;
+  locate_tile(prefix, p.B, p.Hkv, wb, b, kvh, j0);
+  uint32_t qf[NT][KS][2], nq[NT][KS][2];
+  load_q<D, NT>(p, b, kvh, lane, qf);
+  int ctx = clamp_ctx(__ldg(&p.context_lens[b]), cap);
+  bool aborted = false;
+
+  long long t = wb;
+  while (t < we) {
     const int P = prefix[b + 1] - prefix[b];
     const long long seg_first = static_cast<long long>(p.Hkv) * prefix[b] +
                                 static_cast<long long>(kvh) * P;
-    const long long seg_end = min(t_end, seg_first + P);
-    const bool whole = seg_first >= t_begin && seg_first + P <= t_end;
-
-    // query fragments of this group: B operand (Q^T, d x heads), two k-steps per ldmatrix.x4
-    uint32_t qf[NT][KS][2];
-    const int qs = seg_k & 1;
-    // every lane waits (acquire), then the warp agrees so that collective
-    // instructions below run converged even if a wait gave up on some lane
-    const bool qok = __all_sync(0xffffffffu, mbar_wait(&qfull[qs], (seg_k >> 1) & 1, abort_flag));
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int ks = 0; ks < KS; ks += 2) {
-        uint32_t r[4];
-        ldsm_x4(q_base + qs * L::kQTile + sw128_offset(nt * 8 + q_row, ks * 16 + q_col, L::kHeads),
-                r);
-        qf[nt][ks][0] = r[0];
-        qf[nt][ks][1] = r[1];
-        qf[nt][ks + 1][0] = r[2];
-        qf[nt][ks + 1][1] = r[3];
-      }
-    __syncwarp();
-    if (lane == 0 && qok) mbar_arrive(&qempty[qs]);
+    const long long seg_end = min(we, seg_first + P);
+    const bool whole = seg_first >= wb && seg_first + P <= we;
+    // prefetch the next segment's query fragments and length
+    int nb_ = b, nkvh = kvh, nj, nctx = ctx;
+    if (seg_end < we) {
+      locate_tile(prefix, p.B, p.Hkv, seg_end, nb_, nkvh, nj);
+      load_q<D, NT>(p, nb_, nkvh, lane, nq);
+      nctx = clamp_ctx(__ldg(&p.context_lens[nb_]), cap);
+    }
 
     float m[NT][2], l[NT][2], o[KS][NT][4];
 #pragma unroll
@@ -310,16 +369,14 @@ gqa_partition_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int mt = 0; mt < KS; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
     }
 
-    const long long li_first = t - t_begin;
-    const long long li_end = seg_end - t_begin;
-    long long li = li_first + ((cw - static_cast<int>(li_first % kConsumerWarps)) + kConsumerWarps) %
-                                  kConsumerWarps;
-    for (; li < li_end; li += kConsumerWarps) {
-      const int st = static_cast<int>(li % S);
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(&full[st], static_cast<uint32_t>((li / S) & 1), abort_flag)))
-        continue;
-      const int ntok = stage_ntok[st];
+    for (; t < seg_end; ++t) {
+      const long long n = t - wb;
+      const int st = static_cast<int>(n % R);
+      const bool ok = !aborted &&
+          __all_sync(0xffffffffu, mbar_wait(&full[st], static_cast<uint32_t>((n / R) & 1), abort_flag));
+      if (!ok) aborted = true;
+      const int jt = static_cast<int>(t - seg_first);
+      const int ntok = (ok && stage_valid[st]) ? min(kTile, ctx - jt * kTile) : 0;
       if (ntok > 0) {
         const uint32_t kb = ring_base + st * L::kStage;
         const uint32_t vb = kb + L::kKTile;
@@ -395,11 +452,11 @@ gqa_partition_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      __syncwarp();              // every lane is done with this stage
+      if (!aborted) issue_next();
     }
 
-    // ---- combine the four consumer warps' states for this segment
+    // ---- finish the segment (or this warp's piece of it)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -409,56 +466,66 @@ gqa_partition_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int off = 4; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
         l[nt][e] = v;
       }
-    float *cm = comb_me + L::kHeads * L::kCombStride;   // m[kHeads], then l[kHeads]
+    const long long seg = static_cast<long long>(b) * p.Hkv + kvh;
+    const long long slot = gw + seg;
+    uint16_t *orow = reinterpret_cast<uint16_t *>(p.out) +
+                     (static_cast<long long>(b) * p.Hq + kvh * p.G) * D;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int h0 = nt * 8 + 2 * tq;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        const int d0 = mt * 16 + g;
-        comb_me[h0 * L::kCombStride + d0] = o[mt][nt][0];
-        comb_me[(h0 + 1) * L::kCombStride + d0] = o[mt][nt][1];
-        comb_me[h0 * L::kCombStride + d0 + 8] = o[mt][nt][2];
-        comb_me[(h0 + 1) * L::kCombStride + d0 + 8] = o[mt][nt][3];
+      for (int e = 0; e < 2; ++e) {
+        const int h = nt * 8 + 2 * tq + e;
+        if (h >= p.G) continue;
+        const float inv = l[nt][e] > 0.f ? 1.f / l[nt][e] : 0.f;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int d = mt * 16 + g + hf * 8;
+            const float val = o[mt][nt][hf * 2 + e] * inv;
+            if (whole) orow[h * D + d] = to16<BF16>(val);
+            else p.part_o[(slot * p.G + h) * D + d] = val;
+          }
+        if (!whole && g == 0)
+          p.part_lse[slot * p.G + h] = l[nt][e] > 0.f ? m[nt][e] + log2f(l[nt][e]) : -INFINITY;
       }
-      if (g == 0) {
-        cm[h0] = m[nt][0];
-        cm[h0 + 1] = m[nt][1];
-        cm[L::kHeads + h0] = l[nt][0];
-        cm[L::kHeads + h0 + 1] = l[nt][1];
+    if (!whole) {
+      // the last piece of a split segment to finish merges it
+      __syncwarp();
+      const int g0 = piece_of(seg_first, TP, pieces);
+      const int g1 = piece_of(seg_first + P - 1, TP, pieces);
+      int last = 0;
+      if (lane == 0) {
+        int npieces = 0;
+        for (int pc = g0; pc <= g1; ++pc)
+          npieces += piece_begin(pc + 1, TP, pieces) > piece_begin(pc, TP, pieces);
+        __threadfence();
+        last = atomicAdd(&p.seg_count[seg], 1) == npieces - 1;
+        if (last) __threadfence();
       }
+      if (__shfl_sync(0xffffffffu, last, 0))
+        warp_merge<D, BF16>(p.part_o, p.part_lse, orow, p.G, pieces, seg, g0, g1, TP, mstage, lane);
     }
-    named_bar_sync(1, 32 * kConsumerWarps);
-    {
-      const int ct = tid - 32;
-      const long long slot = static_cast<long long>(c) + static_cast<long long>(b) * p.Hkv + kvh;
-      for (int idx = ct; idx < p.G * D; idx += 32 * kConsumerWarps) {
-        const int h = idx / D, d = idx - (idx / D) * D;
-        float M = -INFINITY;
+    // advance to the next segment
+    b = nb_;
+    kvh = nkvh;
+    ctx = nctx;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w)
-          M = fmaxf(M, comb_all[w * (L::kCombWarp / 4) + L::kHeads * L::kCombStride + h]);
-        float acc = 0.f, Ls = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float *cw_base = comb_all + w * (L::kCombWarp / 4);
-          const float mw = cw_base[L::kHeads * L::kCombStride + h];
-          const float a = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-          acc += a * cw_base[h * L::kCombStride + d];
-          Ls += a * cw_base[L::kHeads * L::kCombStride + L::kHeads + h];
-        }
-        const float val = Ls > 0.f ? acc / Ls : 0.f;
-        if (whole) {
-          reinterpret_cast<uint16_t *>(p.out)[(static_cast<long long>(b) * p.Hq + kvh * p.G + h) * D + d] =
-              to16<BF16>(val);
-        } else {
-          p.part_o[(slot * p.G + h) * D + d] = val;
-          if (d == 0) p.part_lse[slot * p.G + h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
-        }
+      for (int ks = 0; ks < KS; ++ks) {
+        qf[nt][ks][0] = nq[nt][ks][0];
+        qf[nt][ks][1] = nq[nt][ks][1];
       }
+  }
+
+  if (aborted && lane == 0) {
+    // leave no copy in flight into shared memory: wait (bounded) for the last R tiles
+    volatile int never = 0;
+    for (long long x = issued > wb + R ? issued - R : wb; x < issued; ++x) {
+      const long long n = x - wb;
+      mbar_wait(&full[n % R], static_cast<uint32_t>((n / R) & 1), &never);
     }
-    named_bar_sync(1, 32 * kConsumerWarps);
-    t = seg_end;
   }
 }
 
