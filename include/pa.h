@@ -34,8 +34,8 @@
  *     Base addresses must be 16-byte aligned.
  *   - workspace is caller-owned device scratch of at least the size returned by
  *     the matching *_workspace_size call; its contents need no initialisation
- *     (pa_decode clears what must start at zero) and are overwritten by every
- *     call.  Two calls in flight at the same time must not share a workspace.
+ *     and are overwritten by every call.  Two calls in flight at the same time
+ *     must not share a workspace.
  *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call is asynchronous on it; nothing is synchronised and no host-side
  *     copy of device data is made.  context_lens and block_table are read only by
@@ -107,40 +107,44 @@ typedef struct {
  * descriptor is invalid or (num_partitions == 0 and no CUDA device is usable). */
 size_t pa_workspace_size(const pa_desc *desc);
 
-/* Full decode step on `stream`: clears the workspace's merge counters, then one
- * fused kernel runs the partition pass and, in the CTA that finishes each split
- * (sequence, kv head) last, the LSE merge of its pieces. */
+/* Full decode step on `stream`: the partition kernel, then the LSE merge kernel
+ * (launched with programmatic dependent launch so that it overlaps the
+ * partition kernel's tail). */
 pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache,
                     const void *v_cache, const int32_t *block_table,
                     const int32_t *context_lens, float scale, void *out, void *workspace,
                     size_t workspace_bytes, void *stream);
 
-/* pa_decode as its two stream operations, for callers that want to time the
- * kernel on its own or reuse one preparation: pa_decode_prepare clears the
- * workspace's per-segment counters (one cudaMemsetAsync, B * Hkv * 4 bytes);
- * pa_decode_launch runs the single fused kernel (partition + LSE merge) and
- * requires a pa_decode_prepare on the same workspace earlier in stream order,
- * with no other pa_decode_launch on that workspace in between. */
-pa_status pa_decode_prepare(const pa_desc *desc, void *workspace, size_t workspace_bytes,
-                            void *stream);
-pa_status pa_decode_launch(const pa_desc *desc, const void *q, const void *k_cache,
-                           const void *v_cache, const int32_t *block_table,
-                           const int32_t *context_lens, float scale, void *out, void *workspace,
-                           size_t workspace_bytes, void *stream);
+/* The two kernels of pa_decode, exposed separately so that each can be timed on
+ * its own: pa_decode_partition runs the partition pass (writes the output of
+ * every (sequence, kv head) that one piece covered, and partials for the rest);
+ * pa_decode_merge combines the partials.  pa_decode_merge must follow
+ * pa_decode_partition on the same stream with the same arguments and workspace. */
+pa_status pa_decode_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                              const void *v_cache, const int32_t *block_table,
+                              const int32_t *context_lens, float scale, void *out,
+                              void *workspace, size_t workspace_bytes, void *stream);
+pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *block_table,
+                          const int32_t *context_lens, float scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream);
 
 size_t pa_mla_workspace_size(const pa_mla_desc *desc);
 
 pa_status pa_decode_mla(const pa_mla_desc *desc, const void *q, const void *latent_cache,
                         const int32_t *block_table, const int32_t *context_lens, float scale,
                         void *out, void *workspace, size_t workspace_bytes, void *stream);
-pa_status pa_decode_mla_prepare(const pa_mla_desc *desc, void *workspace, size_t workspace_bytes,
-                                void *stream);
-pa_status pa_decode_mla_launch(const pa_mla_desc *desc, const void *q, const void *latent_cache,
-                               const int32_t *block_table, const int32_t *context_lens,
-                               float scale, void *out, void *workspace, size_t workspace_bytes,
-                               void *stream);
+pa_status pa_decode_mla_partition(const pa_mla_desc *desc, const void *q,
+                                  const void *latent_cache, const int32_t *block_table,
+                                  const int32_t *context_lens, float scale, void *out,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+pa_status pa_decode_mla_merge(const pa_mla_desc *desc, const void *q, const void *latent_cache,
+                              const int32_t *block_table, const int32_t *context_lens,
+                              float scale, void *out, void *workspace, size_t workspace_bytes,
+                              void *stream);
 
-/* Number of partitions a call with num_partitions == 0 uses on the current
+/* Number of partitions (CTAs of the partition pass; each runs 8 independently
+ * streaming warps, one piece each) a call with num_partitions == 0 uses on the current
  * device (SM count x resident CTAs per SM), or -1 without a usable device.
  * kind: 0 = GQA with this head_dim, 1 = MLA (head_dim ignored). */
 int pa_default_partitions(int kind, int head_dim);

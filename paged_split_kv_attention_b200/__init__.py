@@ -68,14 +68,11 @@ def library() -> ctypes.CDLL:
             vp, sz, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
             gqa = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp, f32, vp, vp, sz, vp]
             mla = [ctypes.POINTER(PAMLADesc), vp, vp, vp, vp, f32, vp, vp, sz, vp]
-            lib.pa_decode.argtypes = gqa
-            lib.pa_decode_launch.argtypes = gqa
-            lib.pa_decode_prepare.argtypes = [ctypes.POINTER(PADesc), vp, sz, vp]
-            lib.pa_decode_mla.argtypes = mla
-            lib.pa_decode_mla_launch.argtypes = mla
-            lib.pa_decode_mla_prepare.argtypes = [ctypes.POINTER(PAMLADesc), vp, sz, vp]
-            for name in ("pa_decode", "pa_decode_launch", "pa_decode_prepare", "pa_decode_mla",
-                         "pa_decode_mla_launch", "pa_decode_mla_prepare"):
+            for name in ("pa_decode", "pa_decode_partition", "pa_decode_merge"):
+                getattr(lib, name).argtypes = gqa
+                getattr(lib, name).restype = ctypes.c_int
+            for name in ("pa_decode_mla", "pa_decode_mla_partition", "pa_decode_mla_merge"):
+                getattr(lib, name).argtypes = mla
                 getattr(lib, name).restype = ctypes.c_int
             lib.pa_workspace_size.argtypes = [ctypes.POINTER(PADesc)]
             lib.pa_workspace_size.restype = sz
@@ -163,16 +160,9 @@ def _workspace(nbytes, device, workspace):
     return workspace
 
 
-_PASSES = {"both": "pa_decode", "launch": "pa_decode_launch"}
-_MLA_PASSES = {"both": "pa_decode_mla", "launch": "pa_decode_mla_launch"}
-
-
-def prepare(desc, workspace, stream=None):
-    """Clear the workspace's merge counters (the first half of a decode step)."""
-    lib = library()
-    fn = lib.pa_decode_prepare if isinstance(desc, PADesc) else lib.pa_decode_mla_prepare
-    _check(fn(ctypes.byref(desc), _ptr(workspace), workspace.numel() * workspace.element_size(),
-              _stream_ptr(stream)), "prepare")
+_PASSES = {"both": "pa_decode", "partition": "pa_decode_partition", "merge": "pa_decode_merge"}
+_MLA_PASSES = {"both": "pa_decode_mla", "partition": "pa_decode_mla_partition",
+               "merge": "pa_decode_mla_merge"}
 
 
 def decode(q, k_cache, v_cache, block_table, context_lens, scale, out=None, workspace=None,
@@ -182,8 +172,8 @@ def decode(q, k_cache, v_cache, block_table, context_lens, scale, out=None, work
     q [B, Hq, D]; k_cache, v_cache [num_blocks, Hkv, block_size, D] (fp16/bf16);
     block_table [B, max_blocks_per_seq] int32; context_lens [B] int32.
     Returns out [B, Hq, D] in q's dtype.  Asynchronous on the current stream.
-    passes="launch" runs only the fused kernel (the workspace must have been
-    cleared by prepare() since its last use).
+    passes="partition" / "merge" run one of the two kernels (merge must follow
+    partition with the same arguments and workspace).
     """
     _require(q, "q", ndim=3)
     _require(k_cache, "k_cache", q.dtype, 4)

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "pa_gqa.cuh"
+#include "pa_merge.cuh"
 #include "pa_mla.cuh"
 
 namespace {
@@ -117,7 +118,7 @@ struct QueryResident {
 
 struct GqaPlan {
   int G = 0, NT = 0, parts = 0;
-  size_t off_cnt = 0, cnt_bytes = 0, off_lse = 0, off_o = 0, bytes = 0;
+  size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
 int default_gqa_parts(int D, int NT, bool bf16, int B) {
@@ -156,9 +157,8 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl) {
   }
   // one partial slot per (warp piece, segment) pair a piece can end: piece + segment
   const size_t slots = size_t(pl->parts) * pa::kWarps + size_t(d->batch) * d->num_kv_heads;
-  pl->off_cnt = 0;
-  pl->cnt_bytes = size_t(d->batch) * d->num_kv_heads * 4;
-  pl->off_lse = round_up(pl->cnt_bytes, 256);
+  pl->off_prefix = 0;
+  pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
   pl->off_o = pl->off_lse + round_up(slots * G * 4, 256);
   pl->bytes = pl->off_o + slots * G * size_t(d->head_dim) * 4;
   return PA_OK;
@@ -192,7 +192,35 @@ struct LaunchPartition {
   }
 };
 
-enum Pass { kPrepare = 1, kLaunch = 2, kBoth = 3 };
+// The merge kernel for value width DV, launched with programmatic dependent
+// launch so that its CTAs can be scheduled while the partition grid drains.
+template <int DV, bool BF16>
+cudaError_t launch_merge(const pa::MergeParams &mp, int segments, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(segments), static_cast<unsigned>(mp.G), 1);
+  cfg.blockDim = dim3(pa::kMergeThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::merge_kernel<DV, BF16>, mp);
+}
+
+cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int segments,
+                           cudaStream_t st) {
+  if (DV == 128) return bf16 ? launch_merge<128, true>(mp, segments, st)
+                             : launch_merge<128, false>(mp, segments, st);
+  if (DV == 64) return bf16 ? launch_merge<64, true>(mp, segments, st)
+                            : launch_merge<64, false>(mp, segments, st);
+  if (DV == 512) return bf16 ? launch_merge<512, true>(mp, segments, st)
+                             : launch_merge<512, false>(mp, segments, st);
+  return cudaErrorInvalidValue;
+}
+
+enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
 
 pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, const void *v,
                   const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
@@ -201,23 +229,15 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
   pa_status s = plan_gqa(d, &pl);
   if (s != PA_OK) return s;
   if (d->batch == 0) return PA_OK;
-  if (passes == kPrepare) {
-    if (!ws || !aligned16(ws) || ws_bytes < pl.bytes) return PA_ERR_WORKSPACE;
-  } else {
-    s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
-    if (s != PA_OK) return s;
-    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-  }
+  s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
+  if (s != PA_OK) return s;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
   const bool bf16 = d->dtype == PA_BF16;
   const int D = d->head_dim;
 
-  if (passes & kPrepare) {
-    // per-segment piece counters of the fused merge start from zero
-    if (cudaMemsetAsync(w + pl.off_cnt, 0, pl.cnt_bytes, st) != cudaSuccess) return PA_ERR_CUDA;
-  }
-  if (passes & kLaunch) {
+  if (passes & kPartition) {
     CUtensorMap maps[2];
     const uint64_t kv_rows = uint64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
     if (!make_map_2d(&maps[0], k, bf16, D, kv_rows, 64, pa::kTile) ||
@@ -230,7 +250,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.out = out;
     p.part_o = reinterpret_cast<float *>(w + pl.off_o);
     p.part_lse = reinterpret_cast<float *>(w + pl.off_lse);
-    p.seg_count = reinterpret_cast<int32_t *>(w + pl.off_cnt);
+    p.prefix_out = reinterpret_cast<int32_t *>(w + pl.off_prefix);
     p.B = d->batch;
     p.Hq = d->num_q_heads;
     p.Hkv = d->num_kv_heads;
@@ -245,6 +265,20 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
     if (err != cudaSuccess) return PA_ERR_CUDA;
+  }
+  if (passes & kMerge) {
+    pa::MergeParams mp;
+    mp.part_o = reinterpret_cast<const float *>(w + pl.off_o);
+    mp.part_lse = reinterpret_cast<const float *>(w + pl.off_lse);
+    mp.prefix = reinterpret_cast<const int32_t *>(w + pl.off_prefix);
+    mp.out = out;
+    mp.B = d->batch;
+    mp.Hq = d->num_q_heads;
+    mp.Hkv = d->num_kv_heads;
+    mp.G = pl.G;
+    mp.pieces = pl.parts * pa::kWarps;
+    if (merge_dispatch(D, bf16, mp, d->batch * d->num_kv_heads, st) != cudaSuccess)
+      return PA_ERR_CUDA;
   }
   return PA_OK;
 }
@@ -268,17 +302,19 @@ pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache, con
                  workspace, workspace_bytes, stream);
 }
 
-pa_status pa_decode_prepare(const pa_desc *desc, void *workspace, size_t workspace_bytes,
-                            void *stream) {
-  return run_gqa(kPrepare, desc, nullptr, nullptr, nullptr, nullptr, nullptr, 1.f, nullptr,
+pa_status pa_decode_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                              const void *v_cache, const int32_t *block_table,
+                              const int32_t *context_lens, float scale, void *out,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+  return run_gqa(kPartition, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
                  workspace, workspace_bytes, stream);
 }
 
-pa_status pa_decode_launch(const pa_desc *desc, const void *q, const void *k_cache,
-                           const void *v_cache, const int32_t *block_table,
-                           const int32_t *context_lens, float scale, void *out, void *workspace,
-                           size_t workspace_bytes, void *stream) {
-  return run_gqa(kLaunch, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *block_table,
+                          const int32_t *context_lens, float scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+  return run_gqa(kMerge, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
                  workspace, workspace_bytes, stream);
 }
 

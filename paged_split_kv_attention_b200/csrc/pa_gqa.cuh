@@ -1,5 +1,5 @@
 // pa_gqa.cuh -- paged split-KV decode for grouped query heads (GQA / MHA / MQA):
-// partition pass and LSE merge in one kernel.
+// the partition pass.
 //
 // What it computes (page "cidian.kuaisou.com: flash decoding ++", snippets on the
 // three Flash-Decoding steps): the KV stream of every (sequence, kv head) is cut
@@ -19,10 +19,10 @@
 // work balances, not at a fixed length.
 //
 // Merge.  A warp that ends a segment it shares with other warps writes its
-// normalised partial and log-sum-exp (slot = warp piece + segment), bumps the
-// segment's counter and, if it is the last of the segment's pieces to finish,
-// merges all of them (they are still in L2) into the output.  Other warps keep
-// streaming meanwhile; no CTA-wide barrier exists after the prologue.
+// normalised partial and log-sum-exp into slot (warp piece + segment); the merge
+// kernel (pa_merge.cuh), launched right behind this one with programmatic
+// dependent launch, combines them.  No barrier, fence or atomic is needed on
+// the streaming path.
 //
 // Data movement (the pages ask that K and V be loaded in parallel as fast as
 // possible, then rescaled and combined).  Each warp is its own pipeline: lane 0
@@ -44,7 +44,6 @@ namespace pa {
 constexpr int kTile = 16;               // tokens per pipeline tile
 constexpr int kWarps = 8;               // independent streaming warps per CTA
 constexpr int kGqaThreads = 32 * kWarps;
-constexpr int kMergeFloats = 256;       // per-warp staging for the merge weights
 
 struct GqaParams {
   const uint16_t *q;            // [B][Hq][D]
@@ -53,7 +52,7 @@ struct GqaParams {
   void *out;                    // [B][Hq][D] 16-bit
   float *part_o;                // [slots][G][D]
   float *part_lse;              // [slots][G], log2 units
-  int32_t *seg_count;           // [B*Hkv] finished pieces per segment, zero at launch
+  int32_t *prefix_out;          // [B+1] tiles per kv head (written by CTA 0 for the merge)
   int B, Hq, Hkv, G, bs, mbs, nb;
   int tiles_per_block;          // bs / 16
   int parts;                    // gridDim.x
@@ -66,8 +65,7 @@ struct GqaLayout {
   static constexpr int kKTile = kTile * D * 2;     // bytes of one K (or V) tile
   static constexpr int kStage = 2 * kKTile;
   static constexpr int ring = 0;                   // warp w: stages [w*R, (w+1)*R)
-  static constexpr int merge = ring + kWarps * R * kStage;
-  static constexpr int bars = merge + kWarps * kMergeFloats * 4;
+  static constexpr int bars = ring + kWarps * R * kStage;
   static constexpr int nbars = kWarps * R;
   static constexpr int info = bars + nbars * 8;     // int stage_valid[kWarps * R]
   static constexpr int flags = info + nbars * 4;    // abort flag + scan scratch
@@ -158,81 +156,6 @@ __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int l
   }
 }
 
-// Third Flash-Decoding step for one split segment, run by the warp that finished
-// the segment last: pieces pc in [g0, g1] left normalised partials o_pc and
-// log-sum-exps lse_pc (log2 units) in slot pc + seg;
-//   out = sum 2^(lse - M) o / sum 2^(lse - M),  M = max lse,
-// with M tracked online over chunks of pieces staged in shared memory.
-template <int D, bool BF16>
-__device__ __noinline__ void warp_merge(const float *part_o, const float *part_lse,
-                                        uint16_t *out_rows, int G, int pieces_total,
-                                        long long seg, int g0, int g1, long long TP,
-                                        float *stage, int lane) {
-  constexpr int F4 = D / 4;                         // float4 per head row
-  const int items = (G * F4 + 31) / 32;              // float4 items per lane
-  const int chunk = kMergeFloats / G;
-  float Mrun[16], Wrun[16];
-  float4 acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    Mrun[i] = -INFINITY;
-    Wrun[i] = 0.f;
-    acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int cs = g0; cs <= g1; cs += chunk) {
-    const int ce = min(g1, cs + chunk - 1);
-    const int n = (ce - cs + 1) * G;
-    for (int i = lane; i < n; i += 32) {
-      const int pc = cs + i / G, h = i - (i / G) * G;
-      stage[i] = piece_begin(pc + 1, TP, pieces_total) > piece_begin(pc, TP, pieces_total)
-                     ? __ldcg(&part_lse[(pc + seg) * G + h])
-                     : -INFINITY;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i >= items) break;
-      const int f = lane + 32 * i;
-      if (f >= G * F4) continue;
-      const int h = f / F4;
-      float Mc = -INFINITY;
-      for (int pc = cs; pc <= ce; ++pc) Mc = fmaxf(Mc, stage[(pc - cs) * G + h]);
-      const float Mn = fmaxf(Mrun[i], Mc);
-      if (Mn == -INFINITY) continue;
-      const float r = Mrun[i] == -INFINITY ? 0.f : exp2f(Mrun[i] - Mn);
-      acc[i].x *= r; acc[i].y *= r; acc[i].z *= r; acc[i].w *= r;
-      Wrun[i] *= r;
-      Mrun[i] = Mn;
-    }
-    for (int pc = cs; pc <= ce; ++pc) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (i >= items) break;
-        const int f = lane + 32 * i;
-        if (f >= G * F4) continue;
-        const int h = f / F4;
-        const float lse = stage[(pc - cs) * G + h];
-        if (lse == -INFINITY) continue;
-        const float w = exp2f(lse - Mrun[i]);
-        const float4 v = __ldcg(reinterpret_cast<const float4 *>(part_o + ((pc + seg) * G) * D) + f);
-        Wrun[i] += w;
-        acc[i].x += w * v.x; acc[i].y += w * v.y; acc[i].z += w * v.z; acc[i].w += w * v.w;
-      }
-    }
-    __syncwarp();
-  }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (i >= items) break;
-    const int f = lane + 32 * i;
-    if (f >= G * F4) continue;
-    const float inv = Wrun[i] > 0.f ? 1.f / Wrun[i] : 0.f;
-    const uint32_t lo = pack2<BF16>(acc[i].x * inv, acc[i].y * inv);
-    const uint32_t hi = pack2<BF16>(acc[i].z * inv, acc[i].w * inv);
-    *reinterpret_cast<uint2 *>(out_rows + static_cast<long long>(f) * 4) = make_uint2(lo, hi);
-  }
-}
-
 template <int D, int NT, bool BF16, int R>
 __global__ void __launch_bounds__(kGqaThreads, 1)
 gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -260,6 +183,10 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + off));
   }
   tiles_prefix<kGqaThreads>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0);
+  if (c == 0)
+    for (int i = tid; i <= p.B; i += kGqaThreads) p.prefix_out[i] = prefix[i];
+  // let the merge grid be scheduled as SMs free up (it waits for this grid to finish)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // sequences with no tokens get an all-zero output row (spread over the grid)
   for (int b = c; b < p.B; b += p.parts)
     if (prefix[b + 1] == prefix[b])
@@ -275,7 +202,6 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::bars) + warp * R;
   int *stage_valid = reinterpret_cast<int *>(sm + L::info) + warp * R;
   uint8_t *ring = sm + L::ring + warp * R * L::kStage;
-  float *mstage = reinterpret_cast<float *>(sm + L::merge) + warp * kMergeFloats;
   if (lane == 0) {
     for (int s = 0; s < R; ++s) mbar_init(&full[s], 1);
     if (warp == 0) *abort_flag = 0;
@@ -489,23 +415,6 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (!whole && g == 0)
           p.part_lse[slot * p.G + h] = l[nt][e] > 0.f ? m[nt][e] + log2f(l[nt][e]) : -INFINITY;
       }
-    if (!whole) {
-      // the last piece of a split segment to finish merges it
-      __syncwarp();
-      const int g0 = piece_of(seg_first, TP, pieces);
-      const int g1 = piece_of(seg_first + P - 1, TP, pieces);
-      int last = 0;
-      if (lane == 0) {
-        int npieces = 0;
-        for (int pc = g0; pc <= g1; ++pc)
-          npieces += piece_begin(pc + 1, TP, pieces) > piece_begin(pc, TP, pieces);
-        __threadfence();
-        last = atomicAdd(&p.seg_count[seg], 1) == npieces - 1;
-        if (last) __threadfence();
-      }
-      if (__shfl_sync(0xffffffffu, last, 0))
-        warp_merge<D, BF16>(p.part_o, p.part_lse, orow, p.G, pieces, seg, g0, g1, TP, mstage, lane);
-    }
     // advance to the next segment
     b = nb_;
     kvh = nkvh;

@@ -14,11 +14,13 @@ pa_status pa_decode_mla(const pa_mla_desc *, const void *, const void *, const i
                         const int32_t *, float, void *, void *, size_t, void *) {
   return PA_ERR_UNSUPPORTED;
 }
-pa_status pa_decode_mla_prepare(const pa_mla_desc *, void *, size_t, void *) {
+pa_status pa_decode_mla_partition(const pa_mla_desc *, const void *, const void *,
+                                  const int32_t *, const int32_t *, float, void *, void *,
+                                  size_t, void *) {
   return PA_ERR_UNSUPPORTED;
 }
-pa_status pa_decode_mla_launch(const pa_mla_desc *, const void *, const void *, const int32_t *,
-                               const int32_t *, float, void *, void *, size_t, void *) {
+pa_status pa_decode_mla_merge(const pa_mla_desc *, const void *, const void *, const int32_t *,
+                              const int32_t *, float, void *, void *, size_t, void *) {
   return PA_ERR_UNSUPPORTED;
 }
 }

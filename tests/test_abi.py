@@ -29,8 +29,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("pa_decode", "pa_decode_mla", "pa_workspace_size", "pa_mla_workspace_size",
-                 "pa_decode_prepare", "pa_decode_launch", "pa_decode_mla_prepare",
-                 "pa_decode_mla_launch", "pa_device_status",
+                 "pa_decode_partition", "pa_decode_merge", "pa_decode_mla_partition",
+                 "pa_decode_mla_merge", "pa_device_status",
                  "pa_status_string"):
         assert want in names, names
 

@@ -147,17 +147,17 @@ def test_long_context_one_sequence(dev):
     assert_close(run_gpu(to_dev(inp, dev), inp["scale"]), ref, "long")
 
 
-def test_prepare_then_launch_equals_full_call(dev):
+def test_partition_then_merge_equals_full_call(dev):
     inp = workloads.make(workloads.get("gqa", batch=5))
     d = to_dev(inp, dev)
     full = run_gpu(d, inp["scale"], num_partitions=37)
     desc = pa().gqa_desc(d["q"], d["k_cache"], d["block_table"], 37)
     ws = torch.full((pa().workspace_size(desc),), 0xAB, dtype=torch.uint8, device=dev)  # garbage
     out = torch.empty_like(d["q"])
-    for _ in range(2):     # twice on one workspace: the counters are re-cleared each time
-        pa().prepare(desc, ws)
-        pa().decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["context_lens"],
-                    inp["scale"], out=out, workspace=ws, num_partitions=37, passes="launch")
+    for _ in range(2):
+        for passes in ("partition", "merge"):
+            pa().decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["context_lens"],
+                        inp["scale"], out=out, workspace=ws, num_partitions=37, passes=passes)
         torch.cuda.synchronize()
         assert torch.equal(out, full)
 
