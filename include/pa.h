@@ -67,7 +67,9 @@ typedef enum {
   PA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, no device) */
   PA_ERR_BAD_BLOCK_ID = 4,  /* device: block id or context length outside the contract */
   PA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out */
-  PA_ERR_WORKSPACE = 6      /* workspace null or smaller than required */
+  PA_ERR_WORKSPACE = 6,     /* workspace null or smaller than required */
+  PA_ERR_TOO_LARGE = 7      /* pa_decode_static: the call needs more scratch than the
+                               library's fixed device buffer holds */
 } pa_status;
 
 typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
@@ -152,6 +154,33 @@ int pa_default_partitions(int kind, int head_dim);
 /* Synchronises `stream`, then returns the first error the kernels recorded on the
  * current device since the last reset (PA_OK if none); reset != 0 clears it. */
 pa_status pa_device_status(void *stream, int reset);
+
+/* pa_decode without a workspace argument, for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is an integration aid.
+ *
+ * Some callers cannot provide scratch: a host runtime that owns all device
+ * memory and lends none to plugins, a serving loop that must never call
+ * cudaMalloc (it can synchronise the device and stall every stream), or a C
+ * program without a caching allocator.  This entry point takes the same inputs
+ * and output as pa_decode and runs the same kernels, but its scratch is a
+ * fixed buffer inside the library: a file-scope device array of
+ * PA_STATIC_SCRATCH_BYTES (16 MiB), present on every GPU that loads the library
+ * until the process exits.  The library allocates nothing here.
+ *
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.  Later calls reuse the address.
+ *   - A call whose workspace (pa_workspace_size) exceeds the buffer returns
+ *     PA_ERR_TOO_LARGE before launching anything.
+ *   - All calls on a device share the one buffer, and it keeps the last call's
+ *     contents.  Nothing in it has to start at zero, so it is never cleared.
+ *     Calls that overlap on the GPU (several streams, or several host threads)
+ *     race on the buffer and corrupt each other's results: serialise them.
+ *   - Errors and asynchrony are as for pa_decode. */
+#define PA_STATIC_SCRATCH_BYTES (16u << 20)
+pa_status pa_decode_static(const pa_desc *desc, const void *q, const void *k_cache,
+                           const void *v_cache, const int32_t *block_table,
+                           const int32_t *context_lens, float scale, void *out, void *stream);
 
 /* Static description of a status code. */
 const char *pa_status_string(pa_status status);

@@ -230,3 +230,31 @@ def device_status(reset: bool = True, stream=None) -> int:
     """Synchronise the stream and return (then clear) the first error the kernels
     recorded on the current device (PA_OK if none)."""
     return int(library().pa_device_status(_stream_ptr(stream), 1 if reset else 0))
+
+
+PA_ERR_TOO_LARGE = 7
+
+
+def decode_static(q, k_cache, v_cache, block_table, context_lens, scale, out=None,
+                  num_partitions=0, stream=None):
+    """pa_decode_static: the same decode with the library's fixed 16 MiB device
+    scratch instead of a caller workspace, for callers that cannot allocate
+    device memory (the output is still the caller's).  Calls that overlap on the
+    GPU share that buffer and must be serialised."""
+    lib = library()
+    fn = lib.pa_decode_static
+    fn.argtypes = [ctypes.POINTER(PADesc)] + [ctypes.c_void_p] * 5 + [ctypes.c_float] + \
+        [ctypes.c_void_p] * 2
+    fn.restype = ctypes.c_int
+    _require(q, "q", ndim=3)
+    _require(k_cache, "k_cache", q.dtype, 4)
+    _require(v_cache, "v_cache", q.dtype, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(context_lens, "context_lens", torch.int32, 1)
+    desc = gqa_desc(q, k_cache, block_table, num_partitions)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(fn(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+              _ptr(context_lens), float(scale), _ptr(out), _stream_ptr(stream)),
+           "pa_decode_static")
+    return out

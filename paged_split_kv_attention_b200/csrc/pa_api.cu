@@ -346,8 +346,54 @@ const char *pa_status_string(pa_status s) {
     case PA_ERR_BAD_BLOCK_ID: return "block id or context length outside the data contract";
     case PA_ERR_TIMEOUT: return "a bounded wait inside a kernel timed out";
     case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_TOO_LARGE: return "call needs more scratch than the static buffer holds";
   }
   return "unknown status";
 }
 
 }  // extern "C"
+
+// ==================================================================== allocation-free entry
+
+// Scratch of pa_decode_static: a fixed device buffer in the library itself, for
+// callers that cannot allocate device memory.  Host code must not pass the
+// symbol itself to a kernel (on the host it names a shadow variable, not device
+// memory); its device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_pa_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device (looked up on the
+// first call per device), or nullptr on error.
+void *static_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_pa_static_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_static_ptr[dev] = ptr;
+  }
+  return g_static_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_static(const pa_desc *desc, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_table,
+                                      const int32_t *context_lens, float scale, void *out,
+                                      void *stream) {
+  GqaPlan pl;
+  pa_status s = plan_gqa(desc, &pl);
+  if (s != PA_OK) return s;
+  if (desc->batch == 0) return PA_OK;
+  if (pl.bytes > PA_STATIC_SCRATCH_BYTES) return PA_ERR_TOO_LARGE;
+  void *scratch = static_scratch_address();
+  if (!scratch) return PA_ERR_CUDA;
+  return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, context_lens, scale, out, scratch,
+                 PA_STATIC_SCRATCH_BYTES, stream);
+}
