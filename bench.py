@@ -218,7 +218,8 @@ def cpu_baseline(w, inp, target_s):
                               nthreads=nthreads)
         return time.perf_counter() - t0
 
-    # calibrate on the first sequence (all heads), then grow to ~target_s
+    # calibrate on the first sequence (all heads), then grow to ~target_s; when the
+    # whole batch takes less than that, repeat whole passes until it is reached
     t1 = max(run(1, H), 1e-4)
     per_tok = t1 / max(int(cl[0]), 1)
     nseq, acc = 0, 0.0
@@ -226,12 +227,15 @@ def cpu_baseline(w, inp, target_s):
         acc += per_tok * int(cl[nseq])
         nseq += 1
     nseq = max(nseq, 1)
-    dt = run(nseq, H)
+    dt, reps = 0.0, 0
+    while reps == 0 or (nseq == w.batch and dt < target_s and reps < 1000):
+        dt += run(nseq, H)
+        reps += 1
     sample_cl = cl[:nseq]
-    nbytes = workloads.kv_bytes(w, sample_cl)
+    nbytes = workloads.kv_bytes(w, sample_cl) * reps
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "sample": f"first {nseq} of {w.batch} sequences ({int(sample_cl.sum())} tokens, all "
-                      f"{H} heads), float64 C oracle, {dt:.2f} s",
+                      f"{H} heads) x {reps} pass(es), float64 C oracle, {dt:.1f} s",
             "seconds": dt}
 
 
