@@ -283,6 +283,141 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
   return PA_OK;
 }
 
+// ------------------------------------------------------------------ MLA
+
+struct MlaPlan {
+  int parts = 0;
+  size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
+};
+
+// CTA pairs that can be resident at once (a pair needs two SMs of one GPC).
+int default_mla_parts() {
+  const size_t smem = pa::MlaLayout::bytes(pa::kMlaMaxBatch);
+  if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  const int sms = sm_count();
+  if (sms < 2) return -1;
+  cfg.gridDim = dim3(static_cast<unsigned>(sms - sms % 2), 1, 1);
+  cfg.blockDim = dim3(pa::kMlaThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, pa::mla_decode_kernel, &cfg) != cudaSuccess ||
+      clusters <= 0)
+    return sms / 2;
+  return clusters;
+}
+
+pa_status plan_mla(const pa_mla_desc *d, MlaPlan *pl) {
+  if (!d) return PA_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->num_heads <= 0 || d->kv_dim <= 0 || d->v_dim <= 0 ||
+      d->block_size <= 0 || d->max_blocks_per_seq <= 0 || d->num_blocks <= 0 ||
+      d->num_partitions < 0 || d->num_partitions > kMaxPartitions)
+    return PA_ERR_INVALID_ARG;
+  if (d->dtype != PA_F16 && d->dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (d->v_dim > d->kv_dim) return PA_ERR_INVALID_ARG;
+  if (d->num_heads != pa::kMlaHeads || d->kv_dim != pa::kMlaDk || d->v_dim != pa::kMlaDv ||
+      d->dtype != PA_BF16)
+    return PA_ERR_UNSUPPORTED;
+  if (d->block_size % pa::kMlaTile || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
+  if (d->batch > pa::kMlaMaxBatch) return PA_ERR_UNSUPPORTED;
+  const int64_t rows = int64_t(d->num_blocks) * d->block_size;
+  const int64_t cap = int64_t(d->max_blocks_per_seq) * d->block_size;
+  if (rows > INT32_MAX || cap > INT32_MAX || int64_t(d->batch) * pa::kMlaHeads > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  pl->parts = d->num_partitions;
+  if (pl->parts == 0) {
+    pl->parts = default_mla_parts();
+    if (pl->parts <= 0) return PA_ERR_CUDA;
+  }
+  const size_t slots = size_t(pl->parts) + size_t(d->batch);
+  pl->off_prefix = 0;
+  pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
+  pl->off_o = pl->off_lse + round_up(slots * pa::kMlaHeads * 4, 256);
+  pl->bytes = pl->off_o + slots * pa::kMlaHeads * size_t(pa::kMlaDv) * 4;
+  return PA_OK;
+}
+
+pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *lat,
+                  const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
+                  size_t ws_bytes, void *stream) {
+  MlaPlan pl;
+  pa_status s = plan_mla(d, &pl);
+  if (s != PA_OK) return s;
+  if (d->batch == 0) return PA_OK;
+  if (!q || !lat || !bt || !cl || !out) return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(lat) || !aligned16(out)) return PA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(bt) & 3u) || (reinterpret_cast<uintptr_t>(cl) & 3u))
+    return PA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < pl.bytes) return PA_ERR_WORKSPACE;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+
+  if (passes & kPartition) {
+    CUtensorMap tq, tl;
+    if (!make_map_2d(&tq, q, true, pa::kMlaDk, uint64_t(d->batch) * pa::kMlaHeads, 64,
+                     pa::kMlaHeads) ||
+        !make_map_2d(&tl, lat, true, pa::kMlaDk, uint64_t(d->num_blocks) * d->block_size, 64,
+                     pa::kMlaTile))
+      return PA_ERR_CUDA;
+    pa::MlaParams p;
+    p.block_table = bt;
+    p.context_lens = cl;
+    p.out = out;
+    p.part_o = reinterpret_cast<float *>(w + pl.off_o);
+    p.part_lse = reinterpret_cast<float *>(w + pl.off_lse);
+    p.prefix_out = reinterpret_cast<int32_t *>(w + pl.off_prefix);
+    p.B = d->batch;
+    p.bs = d->block_size;
+    p.mbs = d->max_blocks_per_seq;
+    p.nb = d->num_blocks;
+    p.tiles_per_block = d->block_size / pa::kMlaTile;
+    p.parts = pl.parts;
+    p.scale_log2 = scale * kLog2e;
+    const size_t smem = pa::MlaLayout::bytes(d->batch);
+    if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return PA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pl.parts), 1, 1);
+    cfg.blockDim = dim3(pa::kMlaThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, tq, tl, p) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  if (passes & kMerge) {
+    pa::MergeParams mp;
+    mp.part_o = reinterpret_cast<const float *>(w + pl.off_o);
+    mp.part_lse = reinterpret_cast<const float *>(w + pl.off_lse);
+    mp.prefix = reinterpret_cast<const int32_t *>(w + pl.off_prefix);
+    mp.out = out;
+    mp.B = d->batch;
+    mp.Hq = pa::kMlaHeads;
+    mp.Hkv = 1;
+    mp.G = pa::kMlaHeads;
+    mp.pieces = pl.parts;
+    if (merge_dispatch(pa::kMlaDv, true, mp, d->batch, st) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -318,12 +453,41 @@ pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cach
                  workspace, workspace_bytes, stream);
 }
 
+size_t pa_mla_workspace_size(const pa_mla_desc *desc) {
+  MlaPlan pl;
+  if (plan_mla(desc, &pl) != PA_OK) return 0;
+  return pl.bytes;
+}
+
+pa_status pa_decode_mla(const pa_mla_desc *desc, const void *q, const void *latent_cache,
+                        const int32_t *block_table, const int32_t *context_lens, float scale,
+                        void *out, void *workspace, size_t workspace_bytes, void *stream) {
+  return run_mla(kBoth, desc, q, latent_cache, block_table, context_lens, scale, out, workspace,
+                 workspace_bytes, stream);
+}
+
+pa_status pa_decode_mla_partition(const pa_mla_desc *desc, const void *q,
+                                  const void *latent_cache, const int32_t *block_table,
+                                  const int32_t *context_lens, float scale, void *out,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+  return run_mla(kPartition, desc, q, latent_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_mla_merge(const pa_mla_desc *desc, const void *q, const void *latent_cache,
+                              const int32_t *block_table, const int32_t *context_lens,
+                              float scale, void *out, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+  return run_mla(kMerge, desc, q, latent_cache, block_table, context_lens, scale, out, workspace,
+                 workspace_bytes, stream);
+}
+
 int pa_default_partitions(int kind, int head_dim) {
   if (kind == 0) {
     if (head_dim != 64 && head_dim != 128) return -1;
     return default_gqa_parts(head_dim, 1, true, 256);
   }
-  return pa_mla_default_parts();
+  return default_mla_parts();
 }
 
 pa_status pa_device_status(void *stream, int reset) {

@@ -1,0 +1,142 @@
+"""GPU parity of the MLA (shared-latent) decode path against the float64 oracle.
+
+128 heads read one 576-wide latent row per token; the value is its first 512
+dims.  Same tolerance as the GQA tests: |gpu - oracle| <= 2e-3 + 1e-2 |oracle|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-3, 1e-2
+
+
+def u16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def pa():
+    import paged_split_kv_attention_b200 as m
+    return m
+
+
+def mla(ctx, seed=0, bs=64, pool="factor:1.3"):
+    return workloads.MLAWorkload("t", len(ctx), 128, 576, 512, "bf16", bs,
+                                 "fixed:" + ",".join(str(c) for c in ctx), pool, seed,
+                                 scale=1.0 / 192 ** 0.5)
+
+
+def ref_of(inp, pairs=None):
+    return oracle.decode_mla(u16(inp["q"]), u16(inp["latent_cache"]), inp["block_table"].numpy(),
+                             inp["context_lens"].numpy(), inp["scale"], inp["dtype"],
+                             v_dim=inp["v_dim"], pairs=pairs)
+
+
+def to_dev(inp, dev):
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+def run(d, inp, **kw):
+    out = pa().decode_mla(d["q"], d["latent_cache"], d["block_table"], d["context_lens"],
+                          inp["scale"], v_dim=inp["v_dim"], **kw)
+    torch.cuda.synchronize()
+    st = pa().device_status()
+    assert st == 0, pa().status_string(st)
+    return out
+
+
+def assert_close(gpu, ref, what=""):
+    g = gpu.float().cpu().numpy().astype(np.float64)
+    err = np.abs(g - ref)
+    bad = err > ATOL + RTOL * np.abs(ref)
+    assert not bad.any(), (f"{what}: {int(bad.sum())}/{bad.size} outside tolerance, "
+                           f"max abs {err.max():.3e}")
+    assert np.isfinite(g).all()
+
+
+@pytest.fixture(scope="module")
+def dev(cuda_device):
+    return cuda_device
+
+
+def test_small_contexts(dev):
+    inp = workloads.make(mla((70, 129), seed=1))
+    ref = ref_of(inp)
+    d = to_dev(inp, dev)
+    for parts in (1, 2, 0):
+        assert_close(run(d, inp, num_partitions=parts), ref, f"parts={parts}")
+
+
+def test_ragged_and_tiny_contexts(dev):
+    inp = workloads.make(mla((1, 64, 65, 0, 127, 300), seed=2))
+    ref = ref_of(inp)
+    d = to_dev(inp, dev)
+    for parts in (1, 3, 7, 0, 50):
+        out = run(d, inp, num_partitions=parts)
+        assert_close(out, ref, f"parts={parts}")
+        assert torch.all(out[3] == 0)
+
+
+@pytest.mark.parametrize("bs", [64, 128])
+def test_block_sizes(dev, bs):
+    inp = workloads.make(mla((200, 1000, 63), seed=3, bs=bs))
+    ref = ref_of(inp)
+    d = to_dev(inp, dev)
+    for parts in (0, 4):
+        assert_close(run(d, inp, num_partitions=parts), ref, f"bs={bs} parts={parts}")
+
+
+def test_scaled_down_mla_workload(dev):
+    inp = workloads.make(workloads.get("mla", batch=3))
+    ref = ref_of(inp)
+    assert_close(run(to_dev(inp, dev), inp), ref, "mla B3")
+
+
+def test_partition_then_merge_equals_full_call(dev):
+    inp = workloads.make(mla((300, 777, 64), seed=4))
+    d = to_dev(inp, dev)
+    full = run(d, inp, num_partitions=5)
+    out = torch.empty_like(full)
+    desc = pa().mla_desc(d["q"], d["latent_cache"], d["block_table"], 512, 5)
+    ws = torch.empty(pa().workspace_size(desc), dtype=torch.uint8, device=dev)
+    for passes in ("partition", "merge"):
+        pa().decode_mla(d["q"], d["latent_cache"], d["block_table"], d["context_lens"],
+                        inp["scale"], v_dim=512, out=out, workspace=ws, num_partitions=5,
+                        passes=passes)
+    torch.cuda.synchronize()
+    assert torch.equal(out, full)
+
+
+def test_repeat_calls_are_bitwise_deterministic(dev):
+    inp = workloads.make(workloads.get("mla", batch=6))
+    d = to_dev(inp, dev)
+    assert torch.equal(run(d, inp), run(d, inp))
+
+
+def test_out_of_range_block_id_is_reported(dev):
+    inp = workloads.make(mla((200, 130), seed=5))
+    d = to_dev(inp, dev)
+    bt = d["block_table"].clone()
+    bt[0, 1] = inp["num_blocks"] + 3
+    pa().device_status(reset=True)
+    pa().decode_mla(d["q"], d["latent_cache"], bt, d["context_lens"], inp["scale"], v_dim=512)
+    assert pa().device_status(reset=True) == pa().PA_ERR_BAD_BLOCK_ID
+    assert_close(run(d, inp), ref_of(inp), "after error")
+
+
+@pytest.mark.slow
+def test_full_size_mla_sampled(dev):
+    w = workloads.get("mla")
+    inp = workloads.make(w)
+    out = run(to_dev(inp, dev), inp)
+    g = torch.Generator().manual_seed(0)
+    cl = inp["context_lens"]
+    bs_ = [int(cl.argmax()), int(cl.argmin())] + torch.randint(0, w.batch, (30,), generator=g).tolist()
+    hs = torch.randint(0, 128, (32,), generator=g).tolist()
+    pairs = np.array(list(zip(bs_, hs)), np.int32)
+    ref = ref_of(inp, pairs=pairs)
+    assert_close(out[pairs[:, 0], pairs[:, 1]], ref, "mla full")
