@@ -100,6 +100,15 @@ def sum_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def rank_workload(name, rank, world):
+    """The workload a rank decodes: the same shapes on every rank, its own seeded
+    batch of independent sequences when several ranks run (weak scaling)."""
+    w = workloads.get(name)
+    if world > 1:
+        w = workloads.get(name, seed=w.seed + 7919 * rank)
+    return w
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -245,9 +254,7 @@ def run_ours(args, rank, world, local):
     import paged_split_kv_attention_b200 as pa
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = workloads.get(args.workload)
-    if world > 1:
-        w = workloads.get(args.workload, seed=w.seed + 7919 * rank)
+    w = rank_workload(args.workload, rank, world)
     inp = workloads.make(w)
     kv_bytes = workloads.kv_bytes(w, inp["context_lens"])
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
