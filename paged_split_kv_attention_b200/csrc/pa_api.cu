@@ -290,30 +290,19 @@ struct MlaPlan {
   size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
-// CTA pairs that can be resident at once (a pair needs two SMs of one GPC).
+// Pieces whose two CTAs can all be resident at once (one CTA per SM).
 int default_mla_parts() {
-  const size_t smem = pa::MlaLayout::bytes(pa::kMlaMaxBatch);
+  const size_t smem = pa::MlaLayout::bytes();
   if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return -1;
-  cudaLaunchConfig_t cfg = {};
   const int sms = sm_count();
-  if (sms < 2) return -1;
-  cfg.gridDim = dim3(static_cast<unsigned>(sms - sms % 2), 1, 1);
-  cfg.blockDim = dim3(pa::kMlaThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, pa::mla_decode_kernel, &cfg) != cudaSuccess ||
-      clusters <= 0)
-    return sms / 2;
-  return clusters;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pa::mla_decode_kernel,
+                                                    pa::kMlaThreads, smem) != cudaSuccess ||
+      per_sm <= 0)
+    per_sm = 1;
+  return sms * per_sm / 2 > 0 ? sms * per_sm / 2 : -1;
 }
 
 pa_status plan_mla(const pa_mla_desc *d, MlaPlan *pl) {
@@ -327,8 +316,7 @@ pa_status plan_mla(const pa_mla_desc *d, MlaPlan *pl) {
   if (d->num_heads != pa::kMlaHeads || d->kv_dim != pa::kMlaDk || d->v_dim != pa::kMlaDv ||
       d->dtype != PA_BF16)
     return PA_ERR_UNSUPPORTED;
-  if (d->block_size % pa::kMlaTile || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
-  if (d->batch > pa::kMlaMaxBatch) return PA_ERR_UNSUPPORTED;
+  if (d->block_size % pa::kMlaBox || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
   const int64_t rows = int64_t(d->num_blocks) * d->block_size;
   const int64_t cap = int64_t(d->max_blocks_per_seq) * d->block_size;
   if (rows > INT32_MAX || cap > INT32_MAX || int64_t(d->batch) * pa::kMlaHeads > INT32_MAX)
@@ -363,13 +351,12 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
   uint8_t *w = static_cast<uint8_t *>(ws);
 
   if (passes & kPartition) {
-    CUtensorMap tq, tl;
-    if (!make_map_2d(&tq, q, true, pa::kMlaDk, uint64_t(d->batch) * pa::kMlaHeads, 64,
-                     pa::kMlaHeads) ||
-        !make_map_2d(&tl, lat, true, pa::kMlaDk, uint64_t(d->num_blocks) * d->block_size, 64,
-                     pa::kMlaTile))
+    CUtensorMap tl;
+    if (!make_map_2d(&tl, lat, true, pa::kMlaDk, uint64_t(d->num_blocks) * d->block_size, 64,
+                     pa::kMlaBox))
       return PA_ERR_CUDA;
     pa::MlaParams p;
+    p.q = static_cast<const uint16_t *>(q);
     p.block_table = bt;
     p.context_lens = cl;
     p.out = out;
@@ -380,10 +367,9 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     p.bs = d->block_size;
     p.mbs = d->max_blocks_per_seq;
     p.nb = d->num_blocks;
-    p.tiles_per_block = d->block_size / pa::kMlaTile;
     p.parts = pl.parts;
     p.scale_log2 = scale * kLog2e;
-    const size_t smem = pa::MlaLayout::bytes(d->batch);
+    const size_t smem = pa::MlaLayout::bytes();
     if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return PA_ERR_CUDA;
@@ -392,14 +378,7 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     cfg.blockDim = dim3(pa::kMlaThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, tq, tl, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, tl, p) != cudaSuccess)
       return PA_ERR_CUDA;
   }
   if (passes & kMerge) {
