@@ -421,34 +421,56 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
     auto load_query = [&](int b) {
       const uint4 *src =
           reinterpret_cast<const uint4 *>(p.q + (static_cast<long long>(b) * kMlaHeads + h) * kMlaDk);
+      // loads in batches of 16 x 16 bytes so that few round trips are serialised
 #pragma unroll 1
-      for (int g = 0; g < kQTmemDims / 64; ++g) {
-        uint32_t v[32];
+      for (int g = 0; g < kQTmemDims / 64; g += 2) {
+        uint4 x[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 x = __ldg(src + g * 8 + i);
-          v[4 * i] = x.x;
-          v[4 * i + 1] = x.y;
-          v[4 * i + 2] = x.z;
-          v[4 * i + 3] = x.w;
+        for (int i = 0; i < 16; ++i) x[i] = __ldg(src + g * 8 + i);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          uint32_t v[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[4 * i] = x[8 * k + i].x;
+            v[4 * i + 1] = x[8 * k + i].y;
+            v[4 * i + 2] = x[8 * k + i].z;
+            v[4 * i + 3] = x[8 * k + i].w;
+          }
+          tmem_st32u(tmem + kTmQ + (g + k) * 32 + lane_off, v);
         }
-        tmem_st32u(tmem + kTmQ + g * 32 + lane_off, v);
       }
       uint8_t *qrow = sm + L::qs + h * 128;
+      constexpr int kQs = L::kQSmemDims / 64;          // 5 slabs: batches of 2, 2, 1
 #pragma unroll 1
-      for (int jq = 0; jq < L::kQSmemDims / 64; ++jq) {
-        uint4 x[8];
+      for (int jq = 0; jq < kQs; jq += 2) {
+        uint4 x[16];
+        const int ns = min(2, kQs - jq);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) x[c] = __ldg(src + kQTmemDims / 8 + jq * 8 + c);
+        for (int i = 0; i < 16; ++i)
+          if (i < 8 * ns) x[i] = __ldg(src + kQTmemDims / 8 + jq * 8 + i);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(qrow + jq * L::kQSlab + ((c ^ (h & 7)) << 4)) = x[c];
+        for (int i = 0; i < 16; ++i)
+          if (i < 8 * ns)
+            *reinterpret_cast<uint4 *>(qrow + (jq + i / 8) * L::kQSlab + (((i & 7) ^ (h & 7)) << 4)) =
+                x[i];
       }
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kQFull]);
+    };
+
+    // Pull the query rows of sequence b into L2 ahead of load_query (fire and
+    // forget: nine 128-byte lines per row).
+    auto prefetch_query = [&](int b) {
+      if (b < 0 || b >= p.B) return;
+      const char *row =
+          reinterpret_cast<const char *>(p.q + (static_cast<long long>(b) * kMlaHeads + h) * kMlaDk);
+#pragma unroll
+      for (int i = 0; i < kMlaDk * 2 / 128; ++i)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(row + i * 128));
     };
 
     // Before the query of the sequence starting at tile m may be written, the
@@ -474,7 +496,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
     float m_run = -INFINITY, l_run = 0.f;
     int ctx = 0;
     // tile 0: its query is needed by the first score MMA
-    if (ntiles > 0) query_for(0);
+    if (ntiles > 0) {
+      prefetch_query(b_first);
+      prefetch_query(b_first + 1);
+      query_for(0);
+    }
     for (int n = 0; n < ntiles; ++n, cur.next()) {
       // S(n+1) can be issued once PV(n-1) is: give it its query now
       if (n + 1 < ntiles) query_for(n + 1);
@@ -485,6 +511,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
         m_run = -INFINITY;
         l_run = 0.f;
         ctx = cur.ctx;
+        if (n > 0) prefetch_query(b + 1);            // the sequence after this one
       }
       const int ntok = min(kMlaTile, ctx - j * kMlaTile);
       const int sb = n % kSBuf;
