@@ -209,8 +209,38 @@ cudaError_t launch_merge(const pa::MergeParams &mp, int segments, cudaStream_t s
   return cudaLaunchKernelEx(&cfg, pa::merge_kernel<DV, BF16>, mp);
 }
 
+// Warp-per-row merge: one warp per (segment, head) row, 8 rows per CTA.
+template <int DV, bool BF16>
+cudaError_t launch_merge_rows(const pa::MergeParams &mp, int segments, cudaStream_t st) {
+  const long long rows = static_cast<long long>(segments) * mp.G;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + pa::kMergeRowsPerCta - 1) / pa::kMergeRowsPerCta),
+                     1, 1);
+  cfg.blockDim = dim3(pa::kMergeRowsPerCta * 32, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::merge_rows_kernel<DV, BF16>, mp);
+}
+
+// Few pieces per segment (short and mixed contexts, MLA): a warp per row keeps
+// every row's loads to two round trips.  Many pieces per segment (one long
+// context spread over the GPU): a CTA per row, whose eight piece groups load in
+// parallel, is faster.
+constexpr int kRowsMergeMaxPieces = 8;
+
 cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int segments,
                            cudaStream_t st) {
+  if (static_cast<long long>(mp.pieces) <= static_cast<long long>(kRowsMergeMaxPieces) * segments) {
+    if (DV == 128) return bf16 ? launch_merge_rows<128, true>(mp, segments, st)
+                               : launch_merge_rows<128, false>(mp, segments, st);
+    if (DV == 512) return bf16 ? launch_merge_rows<512, true>(mp, segments, st)
+                               : launch_merge_rows<512, false>(mp, segments, st);
+  }
   if (DV == 128) return bf16 ? launch_merge<128, true>(mp, segments, st)
                              : launch_merge<128, false>(mp, segments, st);
   if (DV == 64) return bf16 ? launch_merge<64, true>(mp, segments, st)

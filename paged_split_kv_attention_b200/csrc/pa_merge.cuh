@@ -106,3 +106,82 @@ merge_kernel(const MergeParams p) {
 }
 
 }  // namespace pa
+
+namespace pa {
+
+// Warp-per-row form of the same merge: warp w of a CTA merges flattened row
+// r = 8 blockIdx.x + w = segment * G + h.  Lane i fetches the log-sum-exps of
+// pieces g0 + i, g0 + i + 32, ... (one round trip for up to 32 pieces), the warp
+// takes their max, then every lane accumulates float4 columns i, i + 32, ... of
+// the weighted partial rows, four pieces per round so that their loads are in
+// flight together.  No block-level barrier: a CTA's rows finish independently.
+constexpr int kMergeRowsPerCta = 8;
+
+template <int DV, bool BF16>
+__global__ void __launch_bounds__(kMergeRowsPerCta * 32)
+merge_rows_kernel(const MergeParams p) {
+  constexpr int V4 = DV / 128;                   // float4 columns per lane
+  static_assert(V4 * 128 == DV, "DV must be a multiple of 128");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const long long r = static_cast<long long>(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
+  const long long segs = static_cast<long long>(p.B) * p.Hkv;
+  if (r >= segs * p.G) return;
+  const int seg = static_cast<int>(r / p.G), h = static_cast<int>(r - static_cast<long long>(seg) * p.G);
+  const int b = seg / p.Hkv, kvh = seg - (seg / p.Hkv) * p.Hkv;
+  const int P = p.prefix[b + 1] - p.prefix[b];
+  if (P <= 0) return;
+  const long long TP = static_cast<long long>(p.Hkv) * p.prefix[p.B];
+  const long long first = static_cast<long long>(p.Hkv) * p.prefix[b] + static_cast<long long>(kvh) * P;
+  const int g0 = piece_of(first, TP, p.pieces);
+  const int g1 = piece_of(first + P - 1, TP, p.pieces);
+  if (g0 == g1) return;
+
+  // lse of the pieces that own tiles (an empty piece wrote nothing): -inf else
+  auto lse_of = [&](int pc) {
+    if (pc > g1 || piece_begin(pc + 1, TP, p.pieces) == piece_begin(pc, TP, p.pieces))
+      return -INFINITY;
+    return __ldcg(&p.part_lse[(static_cast<long long>(pc) + seg) * p.G + h]);
+  };
+  float l0 = lse_of(g0 + lane);
+  float M = l0;
+  for (int pc = g0 + 32 + lane; pc <= g1; pc += 32) M = fmaxf(M, lse_of(pc));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+
+  float4 acc[V4];
+#pragma unroll
+  for (int k = 0; k < V4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float W = 0.f;
+  for (int base = g0; base <= g1; base += 32) {
+    const float lb = base == g0 ? l0 : lse_of(base + lane);
+    const float wl = lb == -INFINITY ? 0.f : exp2f(lb - M);
+    const int n = min(32, g1 - base + 1);
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+      const float w = __shfl_sync(0xffffffffu, wl, i);
+      if (w == 0.f) continue;                      // empty piece (uniform across the warp)
+      const float4 *row = reinterpret_cast<const float4 *>(
+          p.part_o + ((static_cast<long long>(base + i) + seg) * p.G + h) * DV);
+      W += w;
+#pragma unroll
+      for (int k = 0; k < V4; ++k) {
+        const float4 v = __ldcg(row + lane + 32 * k);
+        acc[k].x += w * v.x;
+        acc[k].y += w * v.y;
+        acc[k].z += w * v.z;
+        acc[k].w += w * v.w;
+      }
+    }
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  uint16_t *o = reinterpret_cast<uint16_t *>(p.out) +
+                (static_cast<long long>(b) * p.Hq + kvh * p.G + h) * DV;
+#pragma unroll
+  for (int k = 0; k < V4; ++k)
+    *reinterpret_cast<uint2 *>(o + 4 * (lane + 32 * k)) =
+        make_uint2(pack2<BF16>(acc[k].x * inv, acc[k].y * inv),
+                   pack2<BF16>(acc[k].z * inv, acc[k].w * inv));
+}
+
+}  // namespace pa
