@@ -156,6 +156,15 @@ int pa_default_partitions(int kind, int head_dim);
  * current device since the last reset (PA_OK if none); reset != 0 clears it. */
 pa_status pa_device_status(void *stream, int reset);
 
+/* Test hook for the kernels' timeout path (not for production use).  While
+ * enabled (process-wide, for GQA calls launched afterwards), one warp of the GQA
+ * partition pass waits on an mbarrier that nothing completes before it issues
+ * any copy; its bounded wait gives up after about one second, records
+ * PA_ERR_TIMEOUT (readable through pa_device_status) and the warp leaves, so the
+ * call's output is incomplete but the CUDA context stays usable.  enable = 0
+ * restores normal operation. */
+void pa_test_inject_stall(int enable);
+
 /* pa_decode without a workspace argument, for callers that cannot allocate
  * device memory.  The pages have no counterpart: this is an integration aid.
  *

@@ -82,6 +82,8 @@ def library() -> ctypes.CDLL:
             lib.pa_default_partitions.restype = ctypes.c_int
             lib.pa_device_status.argtypes = [vp, ctypes.c_int]
             lib.pa_device_status.restype = ctypes.c_int
+            lib.pa_test_inject_stall.argtypes = [ctypes.c_int]
+            lib.pa_test_inject_stall.restype = None
             lib.pa_status_string.argtypes = [ctypes.c_int]
             lib.pa_status_string.restype = ctypes.c_char_p
             _lib = lib
@@ -224,6 +226,12 @@ def decode_mla(q, latent_cache, block_table, context_lens, scale, v_dim=512, out
               _ptr(context_lens), float(scale), _ptr(out), _ptr(ws),
               ws.numel() * ws.element_size(), _stream_ptr(stream)), _MLA_PASSES[passes])
     return out
+
+
+def inject_stall_for_testing(enable: bool) -> None:
+    """Test hook (pa_test_inject_stall): while enabled, GQA partition launches
+    take their bounded-wait timeout path and report PA_ERR_TIMEOUT."""
+    library().pa_test_inject_stall(1 if enable else 0)
 
 
 def device_status(reset: bool = True, stream=None) -> int:

@@ -11,6 +11,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include "pa_gqa.cuh"
@@ -250,6 +251,10 @@ cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int seg
   return cudaErrorInvalidValue;
 }
 
+// Test hook (pa_test_inject_stall): makes the next GQA partition launches take
+// their timeout path.
+std::atomic<int> g_stall_test{0};
+
 enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
 
 pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, const void *v,
@@ -291,6 +296,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.tiles_per_block = d->block_size / pa::kTile;
     p.parts = pl.parts;
     p.scale_log2 = scale * kLog2e;
+    p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     cudaError_t err = cudaSuccess;
     if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
@@ -498,6 +504,8 @@ int pa_default_partitions(int kind, int head_dim) {
   }
   return default_mla_parts();
 }
+
+void pa_test_inject_stall(int enable) { g_stall_test.store(enable ? 1 : 0); }
 
 pa_status pa_device_status(void *stream, int reset) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;

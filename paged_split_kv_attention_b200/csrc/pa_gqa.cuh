@@ -57,6 +57,7 @@ struct GqaParams {
   int tiles_per_block;          // bs / 16
   int parts;                    // gridDim.x
   float scale_log2;             // scale * log2(e)
+  int stall_test;               // test hook: warp 0 of CTA 0 waits on a barrier nothing completes
 };
 
 template <int D, int NT, int R>
@@ -209,6 +210,14 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
   __syncthreads();
   if (wb >= we) return;
+
+  if (p.stall_test && c == 0 && warp == 0) {
+    // Test hook for the timeout path: wait on this warp's first stage barrier
+    // before anything is issued into it, so that nothing can complete the wait.
+    // The bounded wait gives up, records PA_ERR_TIMEOUT and raises the CTA's
+    // abort flag; with no copy in flight the warp simply leaves.
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[0], 0, abort_flag))) return;
+  }
 
   const uint64_t policy = l2_evict_first_policy();
   if (lane == 0) {
