@@ -63,6 +63,9 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", choices=["mha", "mqa"], default=None,
+                    help="sequence-length scaling sweep 512..64k (one JSON line per length)")
+    ap.add_argument("--sweep-batch", type=int, default=1)
     return ap.parse_args()
 
 
@@ -481,8 +484,66 @@ def run_reference(args, rank, world):
         dist.destroy_process_group()
 
 
+def run_sweep(args):
+    """Sequence-length scaling, one JSON line per length: the split decode (default
+    launch, the flattened tile stream cut over every warp of the GPU) beside the
+    same kernel launched with one CTA per 8 (sequence, kv head) segments, i.e. no
+    split across SMs (with 8 or more segments each warp takes one whole segment;
+    with fewer, one CTA's warps share them as a one-block-per-head decode would),
+    the baseline Flash-Decoding is measured against."""
+    import paged_split_kv_attention_b200 as pa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm, _, _, peak_src = measured_peaks()
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    K, W = max(3, min(args.steps, 100)), max(3, args.warmup)
+    for ctx in workloads.SWEEP_CTX:
+        w = workloads.scaling(args.sweep, ctx, args.sweep_batch)
+        inp = workloads.make(w)
+        kv_bytes = workloads.kv_bytes(w, inp["context_lens"])
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        out = torch.empty_like(d["q"])
+        segments = w.batch * w.num_kv_heads
+        res = {}
+        for label, parts in (("split", 0), ("no_split", -(-segments // 8))):
+            desc = pa.gqa_desc(d["q"], d["k_cache"], d["block_table"], parts)
+            ws = torch.empty(pa.workspace_size(desc), dtype=torch.uint8, device=dev)
+            times = []
+            for it in range(W + K):
+                flush_w.zero_()
+                torch.sum(flush_r, dim=0, out=sink)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                pa.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["context_lens"],
+                          inp["scale"], out=out, workspace=ws, num_partitions=parts)
+                e1.record(stream)
+                if it >= W:
+                    times.append((e0, e1))
+            torch.cuda.synchronize()
+            if pa.device_status() != 0:
+                raise RuntimeError("kernel reported an error")
+            us = statistics.median(a.elapsed_time(b) for a, b in times) * 1e3
+            res[label] = {"us_per_step": round(us, 2), "GB/s": round(kv_bytes / us / 1e3, 1),
+                          "frac": round(kv_bytes / us / 1e3 / hbm, 4),
+                          "partitions": parts or pa.default_partitions("gqa", 128)}
+        print(json.dumps({
+            "metric": METRIC, "sweep": args.sweep, "ctx": ctx, "batch": w.batch,
+            "heads": {"q": w.num_q_heads, "kv": w.num_kv_heads, "dim": w.head_dim},
+            "kv_bytes": kv_bytes, "split": res["split"], "no_split": res["no_split"],
+            "speedup_split_vs_no_split": round(res["no_split"]["us_per_step"] /
+                                               res["split"]["us_per_step"], 2),
+            "peak": {"hbm_gbs": hbm, "source": peak_src}, "steps": K, "warmup": W,
+            "l2": "flushed before every step", "data": "synthetic (seeded N(0,1))"}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         run_reference(args, rank, world)

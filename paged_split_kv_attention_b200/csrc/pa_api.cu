@@ -251,6 +251,17 @@ cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int seg
   return cudaErrorInvalidValue;
 }
 
+// An automatic launch (num_partitions == 0) sizes its grid for a full GPU but
+// does not cut a short tile stream into pieces much smaller than the partial
+// output each piece writes: a piece leaves G x D fp32 (GQA: one 16-token K+V tile
+// is 16 x D x 4 bytes, so G tiles per piece keep partials at or below the KV
+// bytes read; at least 2) or 128 x 512 fp32 (MLA: 16 tiles of 64 tokens).  A
+// single short sequence or a single kv head would otherwise spend more on
+// partials and their merge than on the KV.  An explicit partition count is used
+// as given.
+int min_tiles_gqa(int G) { return G > 2 ? G : 2; }
+constexpr int kMinTilesMla = 16;
+
 // Test hook (pa_test_inject_stall): makes the next GQA partition launches take
 // their timeout path.
 std::atomic<int> g_stall_test{0};
@@ -297,6 +308,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.parts = pl.parts;
     p.scale_log2 = scale * kLog2e;
     p.stall_test = g_stall_test.load(std::memory_order_relaxed);
+    p.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
     cudaError_t err = cudaSuccess;
     if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
@@ -313,6 +325,8 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     mp.Hkv = d->num_kv_heads;
     mp.G = pl.G;
     mp.pieces = pl.parts * pa::kWarps;
+    mp.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
+    mp.floor_pieces = static_cast<long long>(pa::kWarps) * d->batch * d->num_kv_heads;
     if (merge_dispatch(D, bf16, mp, d->batch * d->num_kv_heads, st) != cudaSuccess)
       return PA_ERR_CUDA;
   }
@@ -404,6 +418,7 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     p.mbs = d->max_blocks_per_seq;
     p.nb = d->num_blocks;
     p.parts = pl.parts;
+    p.min_tiles = d->num_partitions == 0 ? kMinTilesMla : 0;
     p.scale_log2 = scale * kLog2e;
     const size_t smem = pa::MlaLayout::bytes();
     if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -428,6 +443,8 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     mp.Hkv = 1;
     mp.G = pa::kMlaHeads;
     mp.pieces = pl.parts;
+    mp.min_tiles = d->num_partitions == 0 ? kMinTilesMla : 0;
+    mp.floor_pieces = d->batch;
     if (merge_dispatch(pa::kMlaDv, true, mp, d->batch, st) != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;

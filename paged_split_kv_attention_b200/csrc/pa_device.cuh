@@ -213,6 +213,21 @@ __device__ __forceinline__ long long piece_begin(long long c, long long total, l
   return (c * total) / parts;
 }
 
+// Pieces actually used out of `parts` launched.  With min_units > 0 (an
+// automatic launch) a short stream is not cut finer than min_units per piece,
+// so that partial outputs and their merge stay small next to the work itself,
+// but into at least floor_pieces pieces, so that a short stream still spreads
+// over several warps; with min_units == 0 (an explicit partition count) every
+// piece is used.  The partition and merge kernels compute it from the same
+// arguments.
+__device__ __forceinline__ int used_pieces(int parts, long long total, int min_units,
+                                           long long floor_pieces) {
+  if (min_units <= 0) return parts;
+  long long want = (total + min_units - 1) / min_units;
+  if (want < floor_pieces) want = floor_pieces;
+  return static_cast<int>(want < 1 ? 1 : (want < parts ? want : parts));
+}
+
 // The piece that owns unit t (0 <= t < total).
 __device__ __forceinline__ int piece_of(long long t, long long total, long long parts) {
   return static_cast<int>(((t + 1) * parts + total - 1) / total - 1);

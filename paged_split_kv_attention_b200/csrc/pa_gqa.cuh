@@ -58,6 +58,7 @@ struct GqaParams {
   int parts;                    // gridDim.x
   float scale_log2;             // scale * log2(e)
   int stall_test;               // test hook: warp 0 of CTA 0 waits on a barrier nothing completes
+  int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
 };
 
 template <int D, int NT, int R>
@@ -195,10 +196,11 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         reinterpret_cast<uint16_t *>(p.out)[static_cast<long long>(b) * p.Hq * D + i] = 0;
 
   const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
-  const int pieces = p.parts * kWarps;
+  const int pieces = used_pieces(p.parts * kWarps, TP, p.min_tiles,
+                                 static_cast<long long>(kWarps) * p.B * p.Hkv);
   const int gw = c * kWarps + warp;                     // this warp's piece
-  const long long wb = piece_begin(gw, TP, pieces);
-  const long long we = piece_begin(gw + 1, TP, pieces);
+  const long long wb = gw < pieces ? piece_begin(gw, TP, pieces) : 0;
+  const long long we = gw < pieces ? piece_begin(gw + 1, TP, pieces) : 0;
 
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::bars) + warp * R;
   int *stage_valid = reinterpret_cast<int *>(sm + L::info) + warp * R;

@@ -30,7 +30,9 @@ struct MergeParams {
   const int32_t *prefix;     // [B + 1] tiles per kv head (written by the partition pass)
   void *out;                 // [B][Hq][DV] 16-bit
   int B, Hq, Hkv, G;
-  int pieces;                // pieces of the partition pass
+  int pieces;                // pieces launched by the partition pass
+  int min_tiles;             // the partition pass's min_tiles and floor of pieces
+  long long floor_pieces;    // (see used_pieces)
 };
 
 constexpr int kMergeThreads = 256;
@@ -52,15 +54,16 @@ merge_kernel(const MergeParams p) {
   const int P = p.prefix[b + 1] - p.prefix[b];
   if (P <= 0 || h >= p.G) return;
   const long long TP = static_cast<long long>(p.Hkv) * p.prefix[p.B];
+  const int pieces = used_pieces(p.pieces, TP, p.min_tiles, p.floor_pieces);
   const long long first = static_cast<long long>(p.Hkv) * p.prefix[b] + static_cast<long long>(kvh) * P;
-  const int g0 = piece_of(first, TP, p.pieces);
-  const int g1 = piece_of(first + P - 1, TP, p.pieces);
+  const int g0 = piece_of(first, TP, pieces);
+  const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
 
   // M = max over the pieces that own tiles (an empty piece wrote nothing)
   float M = -INFINITY;
   for (int pc = g0 + tid; pc <= g1; pc += kMergeThreads)
-    if (piece_begin(pc + 1, TP, p.pieces) > piece_begin(pc, TP, p.pieces))
+    if (piece_begin(pc + 1, TP, pieces) > piece_begin(pc, TP, pieces))
       M = fmaxf(M, __ldcg(&p.part_lse[(pc + seg) * p.G + h]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
@@ -75,7 +78,7 @@ merge_kernel(const MergeParams p) {
   float W = 0.f;
 #pragma unroll 4
   for (int pc = g0 + pg; pc <= g1; pc += PG) {
-    if (piece_begin(pc + 1, TP, p.pieces) == piece_begin(pc, TP, p.pieces)) continue;
+    if (piece_begin(pc + 1, TP, pieces) == piece_begin(pc, TP, pieces)) continue;
     const long long row = (pc + seg) * p.G + h;
     const float w = exp2f(__ldcg(&p.part_lse[row]) - M);
     const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.part_o + row * DV) + f);
@@ -132,14 +135,15 @@ merge_rows_kernel(const MergeParams p) {
   const int P = p.prefix[b + 1] - p.prefix[b];
   if (P <= 0) return;
   const long long TP = static_cast<long long>(p.Hkv) * p.prefix[p.B];
+  const int pieces = used_pieces(p.pieces, TP, p.min_tiles, p.floor_pieces);
   const long long first = static_cast<long long>(p.Hkv) * p.prefix[b] + static_cast<long long>(kvh) * P;
-  const int g0 = piece_of(first, TP, p.pieces);
-  const int g1 = piece_of(first + P - 1, TP, p.pieces);
+  const int g0 = piece_of(first, TP, pieces);
+  const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
 
   // lse of the pieces that own tiles (an empty piece wrote nothing): -inf else
   auto lse_of = [&](int pc) {
-    if (pc > g1 || piece_begin(pc + 1, TP, p.pieces) == piece_begin(pc, TP, p.pieces))
+    if (pc > g1 || piece_begin(pc + 1, TP, pieces) == piece_begin(pc, TP, pieces))
       return -INFINITY;
     return __ldcg(&p.part_lse[(static_cast<long long>(pc) + seg) * p.G + h]);
   };

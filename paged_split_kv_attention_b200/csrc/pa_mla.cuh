@@ -74,6 +74,7 @@ struct MlaParams {
   int32_t *prefix_out;          // [B+1] tiles per sequence, inclusive prefix (CTA 0 writes)
   int B, bs, mbs, nb;
   int parts;                    // pieces (two CTAs each)
+  int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
   float scale_log2;
 };
 
@@ -209,8 +210,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
       total += scan_scratch[i];
     }
     const long long TP = total;
-    tb = piece_begin(pair, TP, p.parts);
-    te = piece_begin(pair + 1, TP, p.parts);
+    const int pieces = used_pieces(p.parts, TP, p.min_tiles, p.B);
+    tb = pair < pieces ? piece_begin(pair, TP, pieces) : 0;
+    te = pair < pieces ? piece_begin(pair + 1, TP, pieces) : 0;
     if (blockIdx.x == 0 && tid == 0) p.prefix_out[0] = 0;
     for (int b = b0; b < b1; ++b) {
       const int P = mla_tiles(__ldg(&p.context_lens[b]), cap);

@@ -81,6 +81,20 @@ WORKLOADS = {
                          "factor:1.0", 1005, max_ctx=32768),
 }
 
+# Sequence-length scaling sweep (the pages' Flash-Decoding microbenchmark: multi-
+# head attention on A100 over sequence lengths 512 to 64k at several batch sizes;
+# they give no head count).  Plain reading: 16 query heads of dim 128, bf16,
+# block size 16, every sequence at the same length; "mha" gives each query head
+# its own KV head, "mqa" shares one KV head among all 16.
+SWEEP_CTX = (512, 1024, 2048, 4096, 8192, 16384, 32768, 65536)
+
+
+def scaling(kind: str, ctx: int, batch: int = 1) -> GQAWorkload:
+    hkv = {"mha": 16, "mqa": 1}[kind]
+    return GQAWorkload(f"{kind}_{ctx}", batch, 16, hkv, 128, "bf16", 16, f"const:{ctx}",
+                       "factor:1.0", 1006, max_ctx=ctx)
+
+
 TORCH_DTYPE = {"f16": torch.float16, "bf16": torch.bfloat16}
 
 
