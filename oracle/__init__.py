@@ -63,12 +63,18 @@ def _load():
             lib.pa_oracle_decode.argtypes = [i] * 8 + [p16, p16, p16, p32, p32, d, p32, i, pf64, i]
             lib.pa_oracle_decode_split.argtypes = [i] * 8 + [p16, p16, p16, p32, p32, d, i, pf64, i]
             lib.pa_oracle_decode_mla.argtypes = [i] * 8 + [p16, p16, p32, p32, d, p32, i, pf64, i]
-            for f in (lib.pa_oracle_decode, lib.pa_oracle_decode_split, lib.pa_oracle_decode_mla):
+            p8 = ctypes.POINTER(ctypes.c_uint8)
+            lib.pa_oracle_decode_kv8.argtypes = [i] * 8 + [p16, p8, p8, d, d, p32, p32, d, p32, i,
+                                                           pf64, i]
+            for f in (lib.pa_oracle_decode, lib.pa_oracle_decode_split, lib.pa_oracle_decode_mla,
+                      lib.pa_oracle_decode_kv8):
                 f.restype = ctypes.c_int
             lib.pa_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
             lib.pa_oracle_f16_to_f64.restype = ctypes.c_double
             lib.pa_oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
             lib.pa_oracle_bf16_to_f64.restype = ctypes.c_double
+            lib.pa_oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+            lib.pa_oracle_e4m3_to_f64.restype = ctypes.c_double
             lib.pa_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -140,6 +146,43 @@ def decode(q, k_cache, v_cache, block_table, context_lens, scale, dtype, pairs=N
                               _ptr(cl, ctypes.c_int32), float(scale),
                               None if pp is None else _ptr(pp, ctypes.c_int32), npairs,
                               _ptr(out, ctypes.c_double), int(nthreads))
+    _check(rc)
+    return out
+
+
+def e4m3_to_f64(code: int) -> float:
+    return _load().pa_oracle_e4m3_to_f64(code)
+
+
+def decode_kv8(q, k_cache, v_cache, k_scale, v_scale, block_table, context_lens, scale, dtype,
+               pairs=None, nthreads=0):
+    """Paged GQA decode in float64 over a float8 (E4M3) KV cache.
+
+    q [B,Hq,D] raw 16-bit of `dtype`; k_cache/v_cache [NB,Hkv,bs,D] uint8 E4M3 codes;
+    key = code * k_scale, value = code * v_scale.  Returns float64 [B,Hq,D], or
+    [len(pairs), D] when a list of (b, h) pairs is given.
+    """
+    lib = _load()
+    q = _u16(q)
+    k = np.ascontiguousarray(k_cache, dtype=np.uint8)
+    v = np.ascontiguousarray(v_cache, dtype=np.uint8)
+    bt, cl = _i32(block_table), _i32(context_lens)
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k.shape
+    assert D2 == D and v.shape == k.shape and bt.shape[0] == B and cl.shape == (B,)
+    if pairs is None:
+        out = np.empty((B, Hq, D), np.float64)
+        pp, npairs = None, 0
+    else:
+        pp = _i32(pairs).reshape(-1, 2)
+        npairs = pp.shape[0]
+        out = np.empty((npairs, D), np.float64)
+    rc = lib.pa_oracle_decode_kv8(B, Hq, Hkv, D, bs, bt.shape[1], NB, _dtype_code(dtype),
+                                  _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint8),
+                                  _ptr(v, ctypes.c_uint8), float(k_scale), float(v_scale),
+                                  _ptr(bt, ctypes.c_int32), _ptr(cl, ctypes.c_int32), float(scale),
+                                  None if pp is None else _ptr(pp, ctypes.c_int32), npairs,
+                                  _ptr(out, ctypes.c_double), int(nthreads))
     _check(rc)
     return out
 

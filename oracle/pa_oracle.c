@@ -47,7 +47,8 @@
  *     an all-zero output row.
  *
  * All arithmetic is IEEE double.  Inputs are raw 16-bit patterns (binary16 or
- * bfloat16) decoded exactly to double by the two routines below.
+ * bfloat16) or, for a float8 KV cache, E4M3 bytes, decoded exactly to double by
+ * the routines below.
  */
 #include <math.h>
 #include <stdint.h>
@@ -92,6 +93,24 @@ double pa_oracle_bf16_to_f64(uint16_t h) {
 }
 
 /* Record a failure code from inside a parallel loop (any non-zero code wins). */
+/*
+ * 8-bit float E4M3 (the OCP 8-bit floating point format's E4M3 encoding): 1 sign
+ * bit, 4 exponent bits (bias 7), 3 fraction bits; exponent 0 holds subnormals
+ * m x 2^-9; there is no infinity, and the one pattern with exponent 15 and
+ * fraction 7 is NaN (so the largest finite magnitude is 1.75 x 2^8 = 448).
+ * The pages only name FP8 as a Hopper capability (page "bjpcjp.github.io:
+ * llms-attention", FlashAttention-3 teaser: FP8 low precision); this standard
+ * encoding with one scale per tensor is the plainest reading of an FP8 KV cache.
+ */
+double pa_oracle_e4m3_to_f64(uint8_t c) {
+  const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);
+  else v = ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
 static void set_status(int *status, int code) {
 #ifdef _OPENMP
 #pragma omp atomic write
@@ -176,6 +195,59 @@ int pa_oracle_decode(int B, int Hq, int Hkv, int D, int bs, int mbs, int nb, int
       for (int d = 0; d < D; ++d) {
         acc += qd[d] * decode16(k_cache[row + d], dtype);
         V[(long)t * D + d] = decode16(v_cache[row + d], dtype);
+      }
+      s[t] = scale * acc;
+    }
+    if (bad) set_status(&status, PA_ORACLE_BAD_BLOCK);
+    else softmax_mix(n, s, V, D, o);
+    free(qd); free(s); free(V);
+  }
+  return status;
+}
+
+/*
+ * GQA / MHA / MQA paged decode over a float8 KV cache: k_cache / v_cache hold E4M3
+ * codes (one byte each, layout as pa_oracle_decode) and the key / value is the
+ * decoded code times k_scale / v_scale; q is raw 16-bit of q_dtype.  Otherwise the
+ * same definition as pa_oracle_decode (output [npairs or B*Hq][D] double).
+ */
+int pa_oracle_decode_kv8(int B, int Hq, int Hkv, int D, int bs, int mbs, int nb, int q_dtype,
+                         const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                         double k_scale, double v_scale, const int32_t *block_table,
+                         const int32_t *context_lens, double scale, const int32_t *pairs,
+                         int npairs, double *out, int nthreads) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0 || mbs < 0 || nb < 0)
+    return PA_ORACLE_BAD_ARG;
+  const int G = Hq / Hkv;
+  const long n_out = pairs ? (long)npairs : (long)B * Hq;
+  int status = PA_ORACLE_OK;
+#ifdef _OPENMP
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+  for (long i = 0; i < n_out; ++i) {
+    int b = pairs ? pairs[2 * i] : (int)(i / Hq);
+    int h = pairs ? pairs[2 * i + 1] : (int)(i % Hq);
+    double *o = out + i * D;
+    if (b < 0 || b >= B || h < 0 || h >= Hq) { set_status(&status, PA_ORACLE_BAD_ARG); continue; }
+    int n = context_lens[b];
+    if (n < 0 || (long)n > (long)mbs * bs) { set_status(&status, PA_ORACLE_BAD_ARG); continue; }
+    if (n == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+    int g = h / G;
+    double *qd = malloc(sizeof(double) * D);
+    double *s = malloc(sizeof(double) * n);
+    double *V = malloc(sizeof(double) * (size_t)n * D);
+    if (!qd || !s || !V) { free(qd); free(s); free(V); set_status(&status, PA_ORACLE_NO_MEMORY); continue; }
+    for (int d = 0; d < D; ++d) qd[d] = decode16(q[((long)b * Hq + h) * D + d], q_dtype);
+    int bad = 0;
+    for (int t = 0; t < n; ++t) {
+      long blk = block_of(block_table, mbs, nb, bs, b, t);
+      if (blk < 0) { bad = 1; break; }
+      long row = ((blk * Hkv + g) * bs + t % bs) * (long)D;
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) {
+        acc += qd[d] * (pa_oracle_e4m3_to_f64(k_cache[row + d]) * k_scale);
+        V[(long)t * D + d] = pa_oracle_e4m3_to_f64(v_cache[row + d]) * v_scale;
       }
       s[t] = scale * acc;
     }

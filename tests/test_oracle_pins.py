@@ -273,3 +273,58 @@ def test_mla_equals_single_kv_head_gqa_on_the_latent():
     ref = oracle.decode(u16(inp["q"]), u16(kv), u16(kv), inp["block_table"].numpy(),
                         inp["context_lens"].numpy(), 0.2, "bf16")
     assert np.array_equal(out, ref[:, :, :16])
+
+
+# ---------------------------------------------------------------- float8 KV cache
+
+def test_e4m3_decoding_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = np.array([oracle.e4m3_to_f64(int(c)) for c in codes])
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert list(codes[nan]) == [0x7F, 0xFF]
+    assert np.isnan(mine[nan]).all()
+    assert np.array_equal(mine[~nan], ref[~nan])
+    assert np.nanmax(mine) == 448.0 and oracle.e4m3_to_f64(1) == 2.0 ** -9
+
+
+def _kv8_inputs(seed=0, ctx=(5, 9, 1, 17)):
+    w = workloads.GQAWorkload("t", len(ctx), 4, 2, 16, "bf16", 4,
+                              "fixed:" + ",".join(str(c) for c in ctx), "factor:1.3", seed,
+                              kv_dtype="e4m3")
+    return workloads.make(w)
+
+
+def _run_kv8(inp, k_scale=None, v_scale=None, scale=None):
+    return oracle.decode_kv8(u16(inp["q"]), inp["k_cache"].numpy(), inp["v_cache"].numpy(),
+                             inp["k_scale"] if k_scale is None else k_scale,
+                             inp["v_scale"] if v_scale is None else v_scale,
+                             inp["block_table"].numpy(), inp["context_lens"].numpy(),
+                             inp["scale"] if scale is None else scale, inp["dtype"])
+
+
+def test_kv8_decode_equals_16bit_decode_of_the_dequantised_cache():
+    # code x 2^-6 is exact in bfloat16 (3 fraction bits, exponent well in range),
+    # so the float8 path must reproduce the pinned 16-bit definition bit for bit
+    inp = _kv8_inputs()
+    deq = lambda c: (c.view(torch.float8_e4m3fn).to(torch.float64) * inp["k_scale"])  # noqa: E731
+    k16 = deq(inp["k_cache"]).to(torch.bfloat16)
+    v16 = deq(inp["v_cache"]).to(torch.bfloat16)
+    assert torch.equal(k16.to(torch.float64), deq(inp["k_cache"]))
+    ref = oracle.decode(u16(inp["q"]), u16(k16), u16(v16), inp["block_table"].numpy(),
+                        inp["context_lens"].numpy(), inp["scale"], inp["dtype"])
+    assert np.array_equal(_run_kv8(inp), ref)
+
+
+def test_kv8_key_scale_folds_into_the_softmax_scale():
+    inp = _kv8_inputs(seed=1)
+    a = _run_kv8(inp, k_scale=0.37, v_scale=1.0)
+    b = _run_kv8(inp, k_scale=1.0, v_scale=1.0, scale=inp["scale"] * 0.37)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_kv8_value_scale_scales_the_output():
+    inp = _kv8_inputs(seed=2)
+    a = _run_kv8(inp, v_scale=0.37)
+    b = _run_kv8(inp, v_scale=1.0) * 0.37
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)

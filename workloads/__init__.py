@@ -42,6 +42,7 @@ class GQAWorkload:
     seed: int
     scale: Optional[float] = None   # default 1/sqrt(head_dim)
     max_ctx: Optional[int] = None   # capacity bound for the block table (tokens)
+    kv_dtype: Optional[str] = None  # None: as dtype; "e4m3": float8 codes + per-tensor scale
 
     @property
     def kind(self):
@@ -79,7 +80,15 @@ WORKLOADS = {
                        1004, scale=1.0 / math.sqrt(192.0), max_ctx=8192),
     "mixed": GQAWorkload("mixed", 256, 64, 8, 128, "bf16", 16, "loguniform:1,32768",
                          "factor:1.0", 1005, max_ctx=32768),
+    # the GQA decode workload over a float8 KV cache (E4M3 codes, one scale per
+    # tensor): the same shapes and lengths, half the KV bytes
+    "gqa_fp8": GQAWorkload("gqa_fp8", 32, 32, 8, 128, "bf16", 16, "uniform:512,4096",
+                           "factor:1.25", 1007, max_ctx=4096, kv_dtype="e4m3"),
 }
+
+# Float8 KV inputs: N(0,1) values times 2^6 rounded to E4M3 (|x| up to ~6 sigma stays
+# below the format's 448), stored as codes; the key / value is code x 2^-6.
+KV8_SCALE = 1.0 / 64.0
 
 # Sequence-length scaling sweep (the pages' Flash-Decoding microbenchmark: multi-
 # head attention on A100 over sequence lengths 512 to 64k at several batch sizes;
@@ -150,6 +159,17 @@ def build_block_table(context_lens: torch.Tensor, block_size: int, max_blocks: i
     return table
 
 
+def _randn_e4m3(shape, gen, chunk_rows=4096):
+    """N(0,1) float32 draws times 1 / KV8_SCALE rounded to E4M3 codes (uint8)."""
+    out = torch.empty(shape, dtype=torch.uint8)
+    flat = out.view(shape[0], -1)
+    for r in range(0, shape[0], chunk_rows):
+        rows = min(chunk_rows, shape[0] - r)
+        x = torch.randn((rows, flat.shape[1]), generator=gen, dtype=torch.float32) / KV8_SCALE
+        flat[r:r + rows] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out
+
+
 def _randn16(shape, dtype, gen, chunk_rows=4096):
     """N(0,1) float32 draws rounded to a 16-bit type, drawn in row chunks."""
     out = torch.empty(shape, dtype=TORCH_DTYPE[dtype])
@@ -178,9 +198,16 @@ def make(w, context_lens: Optional[torch.Tensor] = None):
     table = build_block_table(cl, w.block_size, mbs, nb, gen)
     if w.kind == "gqa":
         q = _randn16((w.batch, w.num_q_heads, w.head_dim), w.dtype, gen)
-        k = _randn16((nb, w.num_kv_heads, w.block_size, w.head_dim), w.dtype, gen)
-        v = _randn16((nb, w.num_kv_heads, w.block_size, w.head_dim), w.dtype, gen)
+        kv_shape = (nb, w.num_kv_heads, w.block_size, w.head_dim)
         scale = w.scale if w.scale is not None else 1.0 / math.sqrt(w.head_dim)
+        if w.kv_dtype == "e4m3":
+            k, v = _randn_e4m3(kv_shape, gen), _randn_e4m3(kv_shape, gen)
+            return dict(kind="gqa", q=q, k_cache=k, v_cache=v, block_table=table,
+                        context_lens=cl, scale=scale, dtype=w.dtype, kv_dtype="e4m3",
+                        k_scale=KV8_SCALE, v_scale=KV8_SCALE, num_blocks=nb,
+                        max_blocks_per_seq=mbs)
+        k = _randn16(kv_shape, w.dtype, gen)
+        v = _randn16(kv_shape, w.dtype, gen)
         return dict(kind="gqa", q=q, k_cache=k, v_cache=v, block_table=table, context_lens=cl,
                     scale=scale, dtype=w.dtype, num_blocks=nb, max_blocks_per_seq=mbs)
     q = _randn16((w.batch, w.num_heads, w.kv_dim), w.dtype, gen)
@@ -196,7 +223,8 @@ def kv_bytes(w, context_lens: torch.Tensor) -> int:
     latent once because the value is a prefix of it."""
     tokens = int(context_lens.to(torch.int64).sum())
     if w.kind == "gqa":
-        return tokens * w.num_kv_heads * w.head_dim * 2 * 2
+        elem = 1 if w.kv_dtype == "e4m3" else 2
+        return tokens * w.num_kv_heads * w.head_dim * 2 * elem
     return tokens * w.kv_dim * 2
 
 
