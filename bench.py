@@ -49,6 +49,8 @@ DESCRIPTIONS = {
     "long": "long-context GQA decode: B4 Hq32 Hkv8 D128 bf16 bs64 ctx 131072 shuffled",
     "mla": "MLA absorbed decode: B64 H128 latent 576 (V = first 512) bf16 bs64 ctx U[1024,8192]",
     "mixed": "mixed continuous-batching decode: B256 Hq64 Hkv8 D128 bf16 bs16 ctx log-U[1,32768]",
+    "gqa_fp8": "GQA decode over a float8 E4M3 KV cache (one scale per tensor): B32 Hq32 Hkv8 D128 "
+               "bf16 q/out bs16 ctx U[512,4096] pool 1.25x shuffled",
 }
 
 
@@ -207,12 +209,27 @@ def profiled_traffic(workload, kernel_files):
     return e.get("dram_bytes_per_launch")
 
 
-def cpu_baseline(w, inp, target_s):
-    """Time the float64 oracle on a bounded sample (leading sequences of the batch)."""
+def oracle_rows(w, inp, pairs, nthreads):
+    """The float64 oracle on the given (sequence, head) rows of this workload."""
     import numpy as np
 
     import oracle
     u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    bt, cl = inp["block_table"].numpy(), inp["context_lens"].numpy()
+    if w.kind == "gqa" and getattr(w, "kv_dtype", None) == "e4m3":
+        return oracle.decode_kv8(u16(inp["q"]), inp["k_cache"].numpy(), inp["v_cache"].numpy(),
+                                 inp["k_scale"], inp["v_scale"], bt, cl, inp["scale"],
+                                 inp["dtype"], pairs=pairs, nthreads=nthreads)
+    if w.kind == "gqa":
+        return oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]), bt, cl,
+                             inp["scale"], inp["dtype"], pairs=pairs, nthreads=nthreads)
+    return oracle.decode_mla(u16(inp["q"]), u16(inp["latent_cache"]), bt, cl, inp["scale"],
+                             inp["dtype"], w.v_dim, pairs=pairs, nthreads=nthreads)
+
+
+def cpu_baseline(w, inp, target_s):
+    """Time the float64 oracle on a bounded sample (leading sequences of the batch)."""
+    import numpy as np
     nthreads = os.cpu_count() or 1
     cl = inp["context_lens"]
     H = w.num_q_heads if w.kind == "gqa" else w.num_heads
@@ -220,14 +237,7 @@ def cpu_baseline(w, inp, target_s):
     def run(nseq, nheads):
         pairs = np.array([(b, h) for b in range(nseq) for h in range(nheads)], np.int32)
         t0 = time.perf_counter()
-        if w.kind == "gqa":
-            oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
-                          inp["block_table"].numpy(), cl.numpy(), inp["scale"], inp["dtype"],
-                          pairs=pairs, nthreads=nthreads)
-        else:
-            oracle.decode_mla(u16(inp["q"]), u16(inp["latent_cache"]), inp["block_table"].numpy(),
-                              cl.numpy(), inp["scale"], inp["dtype"], w.v_dim, pairs=pairs,
-                              nthreads=nthreads)
+        oracle_rows(w, inp, pairs, nthreads)
         return time.perf_counter() - t0
 
     # calibrate on the first sequence (all heads), then grow to ~target_s; when the
@@ -264,7 +274,23 @@ def run_ours(args, rank, world, local):
     scale = inp["scale"]
     stream = torch.cuda.current_stream(dev)
 
-    if w.kind == "gqa":
+    kv8 = getattr(w, "kv_dtype", None) == "e4m3"
+    if w.kind == "gqa" and kv8:
+        desc = pa.PADesc(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                         d["block_table"].shape[1], d["k_cache"].shape[0],
+                         pa.PA_BF16 if w.dtype == "bf16" else pa.PA_F16, 0)
+        out = torch.empty_like(d["q"])
+
+        def call(passes):
+            # the float8 entry point runs both passes; a partition-only timing
+            # is not exposed for it
+            return pa.decode_kv8(d["q"], d["k_cache"], d["v_cache"], d["block_table"],
+                                 d["context_lens"], scale, inp["k_scale"], inp["v_scale"],
+                                 out=out, workspace=ws)
+        n_kernels = 1
+        kernel_files = ["pa_gqa.cuh", "pa_device.cuh"]
+        kname = "gqa_decode_kernel (float8 KV)"
+    elif w.kind == "gqa":
         desc = pa.gqa_desc(d["q"], d["k_cache"], d["block_table"])
         out = torch.empty_like(d["q"])
         call = lambda passes: pa.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"],  # noqa
@@ -283,8 +309,8 @@ def run_ours(args, rank, world, local):
         kernel_files = ["pa_mla.cuh", "pa_tcgen05.cuh", "pa_device.cuh"]
         kname = "mla_decode_kernel"
     ws = torch.empty(pa.workspace_size(desc), dtype=torch.uint8, device=dev)
-    parts = desc.num_partitions or pa.default_partitions("gqa" if w.kind == "gqa" else "mla",
-                                                         getattr(w, "head_dim", 128))
+    parts = desc.num_partitions or pa.default_partitions(
+        ("gqa_fp8" if kv8 else "gqa") if w.kind == "gqa" else "mla", getattr(w, "head_dim", 128))
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -356,7 +382,11 @@ def run_ours(args, rank, world, local):
                 e0.record(stream)
             for k2, v in host.items():
                 dev_in[k2].copy_(v, non_blocking=True)
-            if w.kind == "gqa":
+            if w.kind == "gqa" and kv8:
+                pa.decode_kv8(dev_in["q"], dev_in["k_cache"], dev_in["v_cache"],
+                              dev_in["block_table"], dev_in["context_lens"], scale,
+                              inp["k_scale"], inp["v_scale"], out=out, workspace=ws)
+            elif w.kind == "gqa":
                 pa.decode(dev_in["q"], dev_in["k_cache"], dev_in["v_cache"], dev_in["block_table"],
                           dev_in["context_lens"], scale, out=out, workspace=ws)
             else:
@@ -427,10 +457,8 @@ def run_reference(args, rank, world):
         return
     import numpy as np
 
-    import oracle
     w = workloads.get(args.workload)
     inp = workloads.make(w)
-    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
     nthreads = os.cpu_count() or 1
     cl = inp["context_lens"]
     H = w.num_q_heads if w.kind == "gqa" else w.num_heads
@@ -440,14 +468,7 @@ def run_reference(args, rank, world):
     def step(nseq):
         pairs = np.array([(b, h) for b in range(nseq) for h in range(H)], np.int32)
         t0 = time.perf_counter()
-        if w.kind == "gqa":
-            oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
-                          inp["block_table"].numpy(), cl.numpy(), inp["scale"], inp["dtype"],
-                          pairs=pairs, nthreads=nthreads)
-        else:
-            oracle.decode_mla(u16(inp["q"]), u16(inp["latent_cache"]), inp["block_table"].numpy(),
-                              cl.numpy(), inp["scale"], inp["dtype"], w.v_dim, pairs=pairs,
-                              nthreads=nthreads)
+        oracle_rows(w, inp, pairs, nthreads)
         return time.perf_counter() - t0
 
     t1 = max(step(1), 1e-4)

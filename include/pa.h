@@ -146,10 +146,29 @@ pa_status pa_decode_mla_merge(const pa_mla_desc *desc, const void *q, const void
                               float scale, void *out, void *workspace, size_t workspace_bytes,
                               void *stream);
 
+/* pa_decode over a float8 KV cache (next step after the 16-bit path: the pages
+ * name FP8 only as a Hopper capability, page "bjpcjp.github.io: llms-attention",
+ * FlashAttention-3 teaser; the encoding is the OCP 8-bit float E4M3: 1 sign, 4
+ * exponent bits with bias 7, 3 fraction bits, no infinity, NaN = 0x7F / 0xFF).
+ *
+ * k_cache / v_cache: E4M3 codes, one byte each, in the layout of pa_decode
+ * ([num_blocks][num_kv_heads][block_size][head_dim]); the key is code x k_scale,
+ * the value code x v_scale (one scale per tensor, finite).  q and out are
+ * desc->dtype (PA_F16 or PA_BF16); the kernel computes in fp16, which holds every
+ * E4M3 value exactly, so a bf16 q must lie within the fp16 range (|q| < 65504).
+ * Supported: head_dim 128, and everything pa_decode supports otherwise.  The
+ * workspace is sized by pa_workspace_size(desc).  Errors as pa_decode. */
+pa_status pa_decode_kv_e4m3(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *context_lens, float scale, float k_scale,
+                            float v_scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
 /* Number of partitions (CTAs of the partition pass; each runs 8 independently
  * streaming warps, one piece each) a call with num_partitions == 0 uses on the current
  * device (SM count x resident CTAs per SM), or -1 without a usable device.
- * kind: 0 = GQA with this head_dim, 1 = MLA (head_dim ignored). */
+ * kind: 0 = GQA with this head_dim, 1 = MLA (head_dim ignored), 2 = GQA over a
+ * float8 KV cache (head_dim 128). */
 int pa_default_partitions(int kind, int head_dim);
 
 /* Synchronises `stream`, then returns the first error the kernels recorded on the

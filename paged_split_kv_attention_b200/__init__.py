@@ -74,6 +74,9 @@ def library() -> ctypes.CDLL:
             for name in ("pa_decode_mla", "pa_decode_mla_partition", "pa_decode_mla_merge"):
                 getattr(lib, name).argtypes = mla
                 getattr(lib, name).restype = ctypes.c_int
+            lib.pa_decode_kv_e4m3.argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp, f32, f32,
+                                              f32, vp, vp, sz, vp]
+            lib.pa_decode_kv_e4m3.restype = ctypes.c_int
             lib.pa_workspace_size.argtypes = [ctypes.POINTER(PADesc)]
             lib.pa_workspace_size.restype = sz
             lib.pa_mla_workspace_size.argtypes = [ctypes.POINTER(PAMLADesc)]
@@ -138,7 +141,9 @@ def workspace_size(desc) -> int:
 
 
 def default_partitions(kind: str = "gqa", head_dim: int = 128) -> int:
-    return int(library().pa_default_partitions(0 if kind == "gqa" else 1, head_dim))
+    """kind: "gqa", "mla" or "gqa_fp8" (GQA over a float8 KV cache)."""
+    code = {"gqa": 0, "mla": 1, "gqa_fp8": 2}[kind]
+    return int(library().pa_default_partitions(code, head_dim))
 
 
 def _require(t, name, dtype=None, ndim=None):
@@ -198,6 +203,45 @@ def decode(q, k_cache, v_cache, block_table, context_lens, scale, out=None, work
     _check(fn(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
               _ptr(context_lens), float(scale), _ptr(out), _ptr(ws),
               ws.numel() * ws.element_size(), _stream_ptr(stream)), _PASSES[passes])
+    return out
+
+
+def decode_kv8(q, k_cache, v_cache, block_table, context_lens, scale, k_scale, v_scale,
+               out=None, workspace=None, num_partitions=0, stream=None):
+    """pa_decode_kv_e4m3: paged GQA/MHA/MQA decode over a float8 KV cache.
+
+    k_cache, v_cache [num_blocks, Hkv, block_size, 128] uint8 holding E4M3 codes;
+    the key is code * k_scale and the value code * v_scale.  q [B, Hq, 128] fp16 or
+    bf16 (bf16 within the fp16 range).  Returns out [B, Hq, 128] in q's dtype.
+    """
+    _require(q, "q", ndim=3)
+    _require(k_cache, "k_cache", torch.uint8, 4)
+    _require(v_cache, "v_cache", torch.uint8, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(context_lens, "context_lens", torch.int32, 1)
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache shapes differ")
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D:
+        raise ValueError(f"head_dim mismatch: q {D}, cache {D2}")
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"dtype {q.dtype} not supported (fp16/bf16)")
+    desc = PADesc(B, Hq, Hkv, D, bs, block_table.shape[1], NB, _DTYPES[q.dtype],
+                  int(num_partitions))
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _require(out, "out", q.dtype, 3)
+    ws_bytes = workspace_size(desc)
+    if ws_bytes == 0:
+        raise PAError(PA_ERR_UNSUPPORTED, "pa_workspace_size")
+    ws = _workspace(ws_bytes, q.device, workspace)
+    _check(library().pa_decode_kv_e4m3(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(block_table), _ptr(context_lens), float(scale),
+                                       float(k_scale), float(v_scale), _ptr(out), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream_ptr(stream)),
+           "pa_decode_kv_e4m3")
     return out
 
 

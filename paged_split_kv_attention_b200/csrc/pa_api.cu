@@ -62,6 +62,20 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t inner, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Float8 KV cache: one byte per element, rows of `inner` bytes.
+bool make_map_2d_u8(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows,
+                    uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -83,36 +97,41 @@ int resident_ctas(const void *kernel, int threads, size_t smem) {
 
 // ------------------------------------------------------------------ GQA variants
 
-template <int D, int NT, bool BF16>
+template <int D, int NT, bool BF16, bool KV8>
 struct GqaVariant {
-  static constexpr int R = D == 128 ? 3 : 6;    // 24 KB ring per warp either way
-  using L = pa::GqaLayout<D, NT, R>;
+  // 24 KB ring per warp at 16 bits; float8: 4 x 4 KB ring + 8 KB of widened tiles
+  static constexpr int R = KV8 ? 4 : (D == 128 ? 3 : 6);
+  using L = pa::GqaLayout<D, NT, R, KV8>;
   static const void *kernel() {
-    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R>);
+    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, KV8>);
   }
   static void launch(int grid, size_t smem, cudaStream_t st, const CUtensorMap &k,
                      const CUtensorMap &v, const pa::GqaParams &p) {
-    pa::gqa_decode_kernel<D, NT, BF16, R><<<grid, pa::kGqaThreads, smem, st>>>(k, v, p);
+    pa::gqa_decode_kernel<D, NT, BF16, R, KV8><<<grid, pa::kGqaThreads, smem, st>>>(k, v, p);
   }
 };
 
-template <template <int, int, bool> class F, typename... A>
-bool dispatch_gqa(int D, int NT, bool bf16, A &&...a) {
-#define PA_CASE(d, nt, b)                        \
-  if (D == d && NT == nt && bf16 == b) {         \
-    F<d, nt, b>::run(static_cast<A &&>(a)...);   \
-    return true;                                 \
+template <template <int, int, bool, bool> class F, typename... A>
+bool dispatch_gqa(int D, int NT, bool bf16, bool kv8, A &&...a) {
+#define PA_CASE(d, nt, b, k8)                               \
+  if (D == d && NT == nt && bf16 == b && kv8 == k8) {       \
+    F<d, nt, b, k8>::run(static_cast<A &&>(a)...);          \
+    return true;                                            \
   }
-  PA_CASE(128, 1, true) PA_CASE(128, 1, false) PA_CASE(128, 2, true) PA_CASE(128, 2, false)
-  PA_CASE(64, 1, true) PA_CASE(64, 1, false) PA_CASE(64, 2, true) PA_CASE(64, 2, false)
+  PA_CASE(128, 1, true, false) PA_CASE(128, 1, false, false)
+  PA_CASE(128, 2, true, false) PA_CASE(128, 2, false, false)
+  PA_CASE(64, 1, true, false) PA_CASE(64, 1, false, false)
+  PA_CASE(64, 2, true, false) PA_CASE(64, 2, false, false)
+  PA_CASE(128, 1, true, true) PA_CASE(128, 1, false, true)
+  PA_CASE(128, 2, true, true) PA_CASE(128, 2, false, true)
 #undef PA_CASE
   return false;
 }
 
-template <int D, int NT, bool BF16>
+template <int D, int NT, bool BF16, bool KV8>
 struct QueryResident {
   static void run(int B, int *out) {
-    using V = GqaVariant<D, NT, BF16>;
+    using V = GqaVariant<D, NT, BF16, KV8>;
     *out = resident_ctas(V::kernel(), pa::kGqaThreads, V::L::bytes(B));
   }
 };
@@ -122,15 +141,15 @@ struct GqaPlan {
   size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
-int default_gqa_parts(int D, int NT, bool bf16, int B) {
+int default_gqa_parts(int D, int NT, bool bf16, bool kv8, int B) {
   const int sms = sm_count();
   if (sms <= 0) return -1;
   int per = -1;
-  if (!dispatch_gqa<QueryResident>(D, NT, bf16, B, &per) || per <= 0) return -1;
+  if (!dispatch_gqa<QueryResident>(D, NT, bf16, kv8, B, &per) || per <= 0) return -1;
   return sms * per;
 }
 
-pa_status plan_gqa(const pa_desc *d, GqaPlan *pl) {
+pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, bool kv8 = false) {
   if (!d) return PA_ERR_INVALID_ARG;
   if (d->batch < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0 ||
       d->block_size <= 0 || d->max_blocks_per_seq <= 0 || d->num_blocks <= 0 ||
@@ -141,6 +160,7 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl) {
   const int G = d->num_q_heads / d->num_kv_heads;
   if (G > 16) return PA_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (kv8 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (d->block_size % pa::kTile || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
   if (d->batch > kMaxBatch) return PA_ERR_UNSUPPORTED;
   const int64_t kv_rows = int64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
@@ -153,7 +173,7 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl) {
   pl->NT = G <= 8 ? 1 : 2;
   pl->parts = d->num_partitions;
   if (pl->parts == 0) {
-    pl->parts = default_gqa_parts(d->head_dim, pl->NT, d->dtype == PA_BF16, d->batch);
+    pl->parts = default_gqa_parts(d->head_dim, pl->NT, d->dtype == PA_BF16, kv8, d->batch);
     if (pl->parts <= 0) return PA_ERR_CUDA;
   }
   // one partial slot per (warp piece, segment) pair a piece can end: piece + segment
@@ -179,11 +199,11 @@ pa_status check_gqa_args(const pa_desc *d, const GqaPlan &pl, const void *q, con
   return PA_OK;
 }
 
-template <int D, int NT, bool BF16>
+template <int D, int NT, bool BF16, bool KV8>
 struct LaunchPartition {
   static void run(int grid, cudaStream_t st, const CUtensorMap *maps, const pa::GqaParams *p,
                   cudaError_t *err) {
-    using V = GqaVariant<D, NT, BF16>;
+    using V = GqaVariant<D, NT, BF16, KV8>;
     const size_t smem = V::L::bytes(p->B);
     *err = cudaFuncSetAttribute(V::kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(smem));
@@ -268,16 +288,19 @@ std::atomic<int> g_stall_test{0};
 
 enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
 
+// kv8: k / v hold float8 E4M3 codes, key = code x k_scale, value = code x v_scale.
 pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, const void *v,
                   const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
-                  size_t ws_bytes, void *stream) {
+                  size_t ws_bytes, void *stream, bool kv8 = false, float k_scale = 1.f,
+                  float v_scale = 1.f) {
   GqaPlan pl;
-  pa_status s = plan_gqa(d, &pl);
+  pa_status s = plan_gqa(d, &pl, kv8);
   if (s != PA_OK) return s;
   if (d->batch == 0) return PA_OK;
   s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
   if (s != PA_OK) return s;
-  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return PA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
   const bool bf16 = d->dtype == PA_BF16;
@@ -286,9 +309,12 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
   if (passes & kPartition) {
     CUtensorMap maps[2];
     const uint64_t kv_rows = uint64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
-    if (!make_map_2d(&maps[0], k, bf16, D, kv_rows, 64, pa::kTile) ||
-        !make_map_2d(&maps[1], v, bf16, D, kv_rows, 64, pa::kTile))
-      return PA_ERR_CUDA;
+    const bool mapped =
+        kv8 ? make_map_2d_u8(&maps[0], k, D, kv_rows, D, pa::kTile) &&
+                  make_map_2d_u8(&maps[1], v, D, kv_rows, D, pa::kTile)
+            : make_map_2d(&maps[0], k, bf16, D, kv_rows, 64, pa::kTile) &&
+                  make_map_2d(&maps[1], v, bf16, D, kv_rows, 64, pa::kTile);
+    if (!mapped) return PA_ERR_CUDA;
     pa::GqaParams p;
     p.q = static_cast<const uint16_t *>(q);
     p.block_table = bt;
@@ -306,11 +332,12 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.nb = d->num_blocks;
     p.tiles_per_block = d->block_size / pa::kTile;
     p.parts = pl.parts;
-    p.scale_log2 = scale * kLog2e;
+    p.scale_log2 = scale * k_scale * kLog2e;
+    p.v_scale = v_scale;
     p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     p.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
     cudaError_t err = cudaSuccess;
-    if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, pl.parts, st, maps, &p, &err))
+    if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, kv8, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
     if (err != cudaSuccess) return PA_ERR_CUDA;
   }
@@ -459,7 +486,20 @@ extern "C" {
 size_t pa_workspace_size(const pa_desc *desc) {
   GqaPlan pl;
   if (plan_gqa(desc, &pl) != PA_OK) return 0;
-  return pl.bytes;
+  size_t bytes = pl.bytes;
+  GqaPlan pl8;                       // the float8 KV call may launch another grid size
+  if (desc->head_dim == 128 && plan_gqa(desc, &pl8, true) == PA_OK && pl8.bytes > bytes)
+    bytes = pl8.bytes;
+  return bytes;
+}
+
+pa_status pa_decode_kv_e4m3(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *context_lens, float scale, float k_scale,
+                            float v_scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream, true, k_scale, v_scale);
 }
 
 pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache, const void *v_cache,
@@ -517,8 +557,9 @@ pa_status pa_decode_mla_merge(const pa_mla_desc *desc, const void *q, const void
 int pa_default_partitions(int kind, int head_dim) {
   if (kind == 0) {
     if (head_dim != 64 && head_dim != 128) return -1;
-    return default_gqa_parts(head_dim, 1, true, 256);
+    return default_gqa_parts(head_dim, 1, true, false, 256);
   }
+  if (kind == 2) return head_dim == 128 ? default_gqa_parts(128, 1, true, true, 256) : -1;
   return default_mla_parts();
 }
 

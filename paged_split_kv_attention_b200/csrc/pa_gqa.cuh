@@ -35,6 +35,17 @@
 // O^T += V^T P with V^T fragments from ldmatrix.trans and P moved to the B
 // operand layout with movmatrix (as a 16-bit hi + lo pair, two MMAs).  The query
 // fragments of the next segment are prefetched into registers.
+//
+// Float8 KV cache (KV8).  With E4M3 codes in the cache (one key scale and one
+// value scale per tensor; page "bjpcjp.github.io: llms-attention",
+// FlashAttention-3 teaser on FP8 low precision) the ring holds 1-byte tiles
+// (one 16 x 128-byte TMA box for K and one for V), and as soon as a stage lands
+// the warp widens it with cvt.rn.f16x2.e4m3x2 (exact: every E4M3 value is an
+// fp16 value) into a per-warp fp16 tile in the layout the 16-bit path reads,
+// frees the stage for the next copy, and runs the same MMAs in fp16 (a bf16
+// query is converted to fp16 once per segment; it must lie in the fp16 range).
+// The key scale is folded into the softmax scale and the value scale into the
+// final 1 / l, so neither costs anything per token.
 #pragma once
 
 #include "pa_device.cuh"
@@ -59,21 +70,24 @@ struct GqaParams {
   float scale_log2;             // scale * log2(e)
   int stall_test;               // test hook: warp 0 of CTA 0 waits on a barrier nothing completes
   int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
+  float v_scale;                // value scale of a float8 KV cache (1 otherwise)
 };
 
-template <int D, int NT, int R>
+template <int D, int NT, int R, bool KV8 = false>
 struct GqaLayout {
   static constexpr int kHeads = 8 * NT;            // group width padded to the MMA N
-  static constexpr int kKTile = kTile * D * 2;     // bytes of one K (or V) tile
+  static constexpr int kKTile = kTile * D * (KV8 ? 1 : 2);  // bytes of one K (or V) tile
   static constexpr int kStage = 2 * kKTile;
+  static constexpr int kWide = 2 * kTile * D * 2;  // KV8: one widened fp16 K + V tile pair
   static constexpr int ring = 0;                   // warp w: stages [w*R, (w+1)*R)
-  static constexpr int bars = ring + kWarps * R * kStage;
+  static constexpr int wide = ring + kWarps * R * kStage;    // KV8: warp w's fp16 tiles
+  static constexpr int bars = wide + (KV8 ? kWarps * kWide : 0);
   static constexpr int nbars = kWarps * R;
   static constexpr int info = bars + nbars * 8;     // int stage_valid[kWarps * R]
   static constexpr int flags = info + nbars * 4;    // abort flag + scan scratch
   static constexpr int prefix = flags + 64;         // int prefix[B + 1]
   static size_t bytes(int B) { return 1024 + prefix + static_cast<size_t>(B + 1) * 4; }
-  static_assert(kStage % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kStage % 1024 == 0 && wide % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(bars % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
@@ -140,7 +154,23 @@ __device__ __forceinline__ int tile_row(const GqaParams &p, const int *prefix, l
 // Query B-operand fragments (Q^T: d x heads) of group (b, kvh): for n-tile nt and
 // k-step ks, lane holds Q[head 8nt+g][16ks+2tq .. +1] and Q[..][16ks+8+2tq .. +1];
 // heads past the group are zero.
-template <int D, int NT>
+// Two E4M3 codes (low byte = first element) -> an fp16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t r;
+  const uint16_t c = static_cast<uint16_t>(two_codes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(c));
+  return r;
+}
+
+// bf16 pair -> fp16 pair (exact inside the fp16 range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+  const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xffff0000u);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// TO_F16: the query is bf16 and the MMAs run in fp16 (float8 KV cache)
+template <int D, int NT, bool TO_F16 = false>
 __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int lane,
                                        uint32_t (&qf)[NT][D / 16][2]) {
   const int g = lane >> 2, tq = lane & 3;
@@ -154,15 +184,21 @@ __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int l
     for (int ks = 0; ks < D / 16; ++ks) {
       qf[nt][ks][0] = ok ? __ldg(row + ks * 8 + tq) : 0u;
       qf[nt][ks][1] = ok ? __ldg(row + ks * 8 + 4 + tq) : 0u;
+      if (TO_F16) {
+        qf[nt][ks][0] = bf16x2_to_f16x2(qf[nt][ks][0]);
+        qf[nt][ks][1] = bf16x2_to_f16x2(qf[nt][ks][1]);
+      }
     }
   }
 }
 
-template <int D, int NT, bool BF16, int R>
+template <int D, int NT, bool BF16, int R, bool KV8 = false>
 __global__ void __launch_bounds__(kGqaThreads, 1)
 gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
-  using L = GqaLayout<D, NT, R>;
+  using L = GqaLayout<D, NT, R, KV8>;
+  static_assert(!KV8 || D == 128, "the float8 KV path reads 128-byte rows");
+  constexpr bool CT = BF16 && !KV8;          // MMA operand type: bf16, else fp16
   constexpr int KS = D / 16;                 // k-steps of the score MMA / m-tiles of the PV MMA
 
   extern __shared__ uint8_t smem_raw[];
@@ -205,6 +241,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::bars) + warp * R;
   int *stage_valid = reinterpret_cast<int *>(sm + L::info) + warp * R;
   uint8_t *ring = sm + L::ring + warp * R * L::kStage;
+  uint8_t *wide = sm + L::wide + warp * L::kWide;   // KV8 only
   if (lane == 0) {
     for (int s = 0; s < R; ++s) mbar_init(&full[s], 1);
     if (warp == 0) *abort_flag = 0;
@@ -255,11 +292,16 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         stage_valid[st] = 1;
         mbar_arrive_expect_tx(&full[st], L::kStage);
         uint8_t *dst = ring + st * L::kStage;
+        if (KV8) {                                    // one 16 x 128-byte box each
+          tma_load_2d_hint(dst, &tm_k, &full[st], 0, row, policy);
+          tma_load_2d_hint(dst + L::kKTile, &tm_v, &full[st], 0, row, policy);
+        } else {
 #pragma unroll
-        for (int x = 0; x < D; x += 64) {
-          tma_load_2d_hint(dst + (x / 64) * kTile * 128, &tm_k, &full[st], x, row, policy);
-          tma_load_2d_hint(dst + L::kKTile + (x / 64) * kTile * 128, &tm_v, &full[st], x, row,
-                           policy);
+          for (int x = 0; x < D; x += 64) {
+            tma_load_2d_hint(dst + (x / 64) * kTile * 128, &tm_k, &full[st], x, row, policy);
+            tma_load_2d_hint(dst + L::kKTile + (x / 64) * kTile * 128, &tm_v, &full[st], x, row,
+                             policy);
+          }
         }
       }
     }
@@ -278,7 +320,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   int b, kvh, j0;
   locate_tile(prefix, p.B, p.Hkv, wb, b, kvh, j0);
   uint32_t qf[NT][KS][2], nq[NT][KS][2];
-  load_q<D, NT>(p, b, kvh, lane, qf);
+  load_q<D, NT, BF16 && KV8>(p, b, kvh, lane, qf);
   int ctx = clamp_ctx(__ldg(&p.context_lens[b]), cap);
   bool aborted = false;
 
@@ -293,7 +335,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     int nb_ = b, nkvh = kvh, nj, nctx = ctx;
     if (seg_end < we) {
       locate_tile(prefix, p.B, p.Hkv, seg_end, nb_, nkvh, nj);
-      load_q<D, NT>(p, nb_, nkvh, lane, nq);
+      load_q<D, NT, BF16 && KV8>(p, nb_, nkvh, lane, nq);
       nctx = clamp_ctx(__ldg(&p.context_lens[nb_]), cap);
     }
 
@@ -314,9 +356,41 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       if (!ok) aborted = true;
       const int jt = static_cast<int>(t - seg_first);
       const int ntok = (ok && stage_valid[st]) ? min(kTile, ctx - jt * kTile) : 0;
+      uint32_t kb = ring_base + st * L::kStage;
+      if (KV8) {
+        if (ntok > 0) {
+          // widen the landed 1-byte tiles into this warp's fp16 tiles: 16-byte
+          // chunk c16 of row r (swizzled position c16 ^ (r & 7)) -> dims
+          // 16 c16 .. 16 c16 + 15 of row r in the 16-bit layout
+          const uint8_t *src = ring + st * L::kStage;
+          uint8_t *dst = wide;
+#pragma unroll
+          for (int i = 0; i < 2 * kTile * 8 / 32; ++i) {
+            const int q = lane + 32 * i;              // chunk of the K (q < 128) or V tile
+            const int vt = q >> 7, r = (q >> 3) & 15, c16 = q & 7;
+            const uint4 x = *reinterpret_cast<const uint4 *>(
+                src + vt * L::kKTile + r * 128 + ((c16 ^ (r & 7)) << 4));
+            uint4 lo, hi;
+            lo.x = e4m3x2_to_f16x2(x.x & 0xffffu);
+            lo.y = e4m3x2_to_f16x2(x.x >> 16);
+            lo.z = e4m3x2_to_f16x2(x.y & 0xffffu);
+            lo.w = e4m3x2_to_f16x2(x.y >> 16);
+            hi.x = e4m3x2_to_f16x2(x.z & 0xffffu);
+            hi.y = e4m3x2_to_f16x2(x.z >> 16);
+            hi.z = e4m3x2_to_f16x2(x.w & 0xffffu);
+            hi.w = e4m3x2_to_f16x2(x.w >> 16);
+            uint8_t *t = dst + vt * (kTile * D * 2);
+            *reinterpret_cast<uint4 *>(t + sw128_offset(r, c16 * 16, kTile)) = lo;
+            *reinterpret_cast<uint4 *>(t + sw128_offset(r, c16 * 16 + 8, kTile)) = hi;
+          }
+        }
+        __syncwarp();            // the stage is read: refill it now
+        if (!aborted) issue_next();
+        __syncwarp();            // the widened tiles are written
+        kb = smem_u32(wide);
+      }
       if (ntok > 0) {
-        const uint32_t kb = ring_base + st * L::kStage;
-        const uint32_t vb = kb + L::kKTile;
+        const uint32_t vb = kb + (KV8 ? kTile * D * 2 : L::kKTile);
         // S^T (16 tokens x 8NT heads) = K Q^T
         float s[NT][4];
 #pragma unroll
@@ -326,7 +400,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
           uint32_t a[4];
           ldsm_x4(kb + sw128_offset(k_row, ks * 16 + k_col, kTile), a);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_16816<BF16>(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+          for (int nt = 0; nt < NT; ++nt) mma_16816<CT>(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
         }
         // online softmax over the tile's tokens (rows g and g + 8 of this lane)
         const bool v0 = g < ntok, v1 = g + 8 < ntok;
@@ -362,8 +436,8 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
           // ~16 bits: one rounded copy alone would bias the value mix against
           // the fp32 row sum l by up to 2^-9 relative.
           uint32_t h01, l01, h23, l23;
-          split2<BF16>(p0, p1, h01, l01);
-          split2<BF16>(p2, p3, h23, l23);
+          split2<CT>(p0, p1, h01, l01);
+          split2<CT>(p2, p3, h23, l23);
           pb[nt][0] = movmatrix_trans(h01);
           pb[nt][1] = movmatrix_trans(h23);
           pl[nt][0] = movmatrix_trans(l01);
@@ -384,13 +458,13 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
           a[3] &= mhi;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            mma_16816<BF16>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
-            mma_16816<BF16>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+            mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+            mma_16816<CT>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
           }
         }
       }
       __syncwarp();              // every lane is done with this stage
-      if (!aborted) issue_next();
+      if (!KV8 && !aborted) issue_next();
     }
 
     // ---- finish the segment (or this warp's piece of it)
@@ -413,7 +487,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       for (int e = 0; e < 2; ++e) {
         const int h = nt * 8 + 2 * tq + e;
         if (h >= p.G) continue;
-        const float inv = l[nt][e] > 0.f ? 1.f / l[nt][e] : 0.f;
+        const float inv = l[nt][e] > 0.f ? p.v_scale / l[nt][e] : 0.f;
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
