@@ -99,8 +99,8 @@ int resident_ctas(const void *kernel, int threads, size_t smem) {
 
 template <int D, int NT, bool BF16, bool KV8>
 struct GqaVariant {
-  // 24 KB ring per warp at 16 bits; float8: 4 x 4 KB ring + 8 KB of widened tiles
-  static constexpr int R = KV8 ? 4 : (D == 128 ? 3 : 6);
+  // 24 KB ring per warp: 3 x 8 KB (D 128), 6 x 4 KB (D 64 or float8 D 128)
+  static constexpr int R = KV8 ? 6 : (D == 128 ? 3 : 6);
   using L = pa::GqaLayout<D, NT, R, KV8>;
   static const void *kernel() {
     return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, KV8>);

@@ -39,13 +39,16 @@
 // Float8 KV cache (KV8).  With E4M3 codes in the cache (one key scale and one
 // value scale per tensor; page "bjpcjp.github.io: llms-attention",
 // FlashAttention-3 teaser on FP8 low precision) the ring holds 1-byte tiles
-// (one 16 x 128-byte TMA box for K and one for V), and as soon as a stage lands
-// the warp widens it with cvt.rn.f16x2.e4m3x2 (exact: every E4M3 value is an
-// fp16 value) into a per-warp fp16 tile in the layout the 16-bit path reads,
-// frees the stage for the next copy, and runs the same MMAs in fp16 (a bf16
-// query is converted to fp16 once per segment; it must lie in the fp16 range).
-// The key scale is folded into the softmax scale and the value scale into the
-// final 1 / l, so neither costs anything per token.
+// (one 16 x 128-byte TMA box for K and one for V, R = 6 stages).  The fragments
+// are built straight from them: ldmatrix of the codes read as 16-bit pairs hands
+// each lane four consecutive codes of one row (K) or, transposed, two dims x two
+// tokens (V, paired per dim by one byte permute), and cvt.rn.f16x2.e4m3x2 widens
+// them exactly (every E4M3 value is an fp16 value).  This fixes which head dims
+// meet in a fragment: the query fragment takes the same dims, and the output
+// rows are written back in dim order.  The MMAs then run in fp16 (a bf16 query
+// is converted to fp16 once per segment; it must lie in the fp16 range).  The
+// key scale is folded into the softmax scale and the value scale into the final
+// 1 / l, so neither costs anything per token.
 #pragma once
 
 #include "pa_device.cuh"
@@ -78,16 +81,14 @@ struct GqaLayout {
   static constexpr int kHeads = 8 * NT;            // group width padded to the MMA N
   static constexpr int kKTile = kTile * D * (KV8 ? 1 : 2);  // bytes of one K (or V) tile
   static constexpr int kStage = 2 * kKTile;
-  static constexpr int kWide = 2 * kTile * D * 2;  // KV8: one widened fp16 K + V tile pair
   static constexpr int ring = 0;                   // warp w: stages [w*R, (w+1)*R)
-  static constexpr int wide = ring + kWarps * R * kStage;    // KV8: warp w's fp16 tiles
-  static constexpr int bars = wide + (KV8 ? kWarps * kWide : 0);
+  static constexpr int bars = ring + kWarps * R * kStage;
   static constexpr int nbars = kWarps * R;
   static constexpr int info = bars + nbars * 8;     // int stage_valid[kWarps * R]
   static constexpr int flags = info + nbars * 4;    // abort flag + scan scratch
   static constexpr int prefix = flags + 64;         // int prefix[B + 1]
   static size_t bytes(int B) { return 1024 + prefix + static_cast<size_t>(B + 1) * 4; }
-  static_assert(kStage % 1024 == 0 && wide % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kStage % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(bars % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
@@ -154,12 +155,12 @@ __device__ __forceinline__ int tile_row(const GqaParams &p, const int *prefix, l
 // Query B-operand fragments (Q^T: d x heads) of group (b, kvh): for n-tile nt and
 // k-step ks, lane holds Q[head 8nt+g][16ks+2tq .. +1] and Q[..][16ks+8+2tq .. +1];
 // heads past the group are zero.
-// Two E4M3 codes (low byte = first element) -> an fp16 pair (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  uint32_t r;
-  const uint16_t c = static_cast<uint16_t>(two_codes);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(c));
-  return r;
+// Two E4M3 code pairs (bytes 0,1 and bytes 2,3 of x) -> two fp16 pairs, exactly
+// (every E4M3 value is an fp16 value).
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t x, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(x));
 }
 
 // bf16 pair -> fp16 pair (exact inside the fp16 range)
@@ -169,8 +170,12 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// TO_F16: the query is bf16 and the MMAs run in fp16 (float8 KV cache)
-template <int D, int NT, bool TO_F16 = false>
+// TO_F16: the query is bf16 and the MMAs run in fp16 (float8 KV cache).
+// KV8: the float8 path feeds the score MMA's k-step ks with head dims
+// 16 ks + 4 tq + {0, 1} as fragment columns 2 tq, 2 tq + 1 and 16 ks + 4 tq + {2, 3}
+// as columns 2 tq + 8, 2 tq + 9 (the order an 8-bit row arrives in, see the
+// kernel); the query fragment takes the same dims.
+template <int D, int NT, bool TO_F16 = false, bool KV8 = false>
 __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int lane,
                                        uint32_t (&qf)[NT][D / 16][2]) {
   const int g = lane >> 2, tq = lane & 3;
@@ -182,8 +187,8 @@ __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int l
         p.q + (static_cast<long long>(b) * p.Hq + kvh * p.G + (ok ? h : 0)) * D);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      qf[nt][ks][0] = ok ? __ldg(row + ks * 8 + tq) : 0u;
-      qf[nt][ks][1] = ok ? __ldg(row + ks * 8 + 4 + tq) : 0u;
+      qf[nt][ks][0] = ok ? __ldg(row + ks * 8 + (KV8 ? 2 * tq : tq)) : 0u;
+      qf[nt][ks][1] = ok ? __ldg(row + ks * 8 + (KV8 ? 2 * tq + 1 : 4 + tq)) : 0u;
       if (TO_F16) {
         qf[nt][ks][0] = bf16x2_to_f16x2(qf[nt][ks][0]);
         qf[nt][ks][1] = bf16x2_to_f16x2(qf[nt][ks][1]);
@@ -241,7 +246,6 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::bars) + warp * R;
   int *stage_valid = reinterpret_cast<int *>(sm + L::info) + warp * R;
   uint8_t *ring = sm + L::ring + warp * R * L::kStage;
-  uint8_t *wide = sm + L::wide + warp * L::kWide;   // KV8 only
   if (lane == 0) {
     for (int s = 0; s < R; ++s) mbar_init(&full[s], 1);
     if (warp == 0) *abort_flag = 0;
@@ -320,7 +324,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   int b, kvh, j0;
   locate_tile(prefix, p.B, p.Hkv, wb, b, kvh, j0);
   uint32_t qf[NT][KS][2], nq[NT][KS][2];
-  load_q<D, NT, BF16 && KV8>(p, b, kvh, lane, qf);
+  load_q<D, NT, BF16 && KV8, KV8>(p, b, kvh, lane, qf);
   int ctx = clamp_ctx(__ldg(&p.context_lens[b]), cap);
   bool aborted = false;
 
@@ -335,7 +339,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     int nb_ = b, nkvh = kvh, nj, nctx = ctx;
     if (seg_end < we) {
       locate_tile(prefix, p.B, p.Hkv, seg_end, nb_, nkvh, nj);
-      load_q<D, NT, BF16 && KV8>(p, nb_, nkvh, lane, nq);
+      load_q<D, NT, BF16 && KV8, KV8>(p, nb_, nkvh, lane, nq);
       nctx = clamp_ctx(__ldg(&p.context_lens[nb_]), cap);
     }
 
@@ -356,51 +360,46 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       if (!ok) aborted = true;
       const int jt = static_cast<int>(t - seg_first);
       const int ntok = (ok && stage_valid[st]) ? min(kTile, ctx - jt * kTile) : 0;
-      uint32_t kb = ring_base + st * L::kStage;
-      if (KV8) {
-        if (ntok > 0) {
-          // widen the landed 1-byte tiles into this warp's fp16 tiles: 16-byte
-          // chunk c16 of row r (swizzled position c16 ^ (r & 7)) -> dims
-          // 16 c16 .. 16 c16 + 15 of row r in the 16-bit layout
-          const uint8_t *src = ring + st * L::kStage;
-          uint8_t *dst = wide;
-#pragma unroll
-          for (int i = 0; i < 2 * kTile * 8 / 32; ++i) {
-            const int q = lane + 32 * i;              // chunk of the K (q < 128) or V tile
-            const int vt = q >> 7, r = (q >> 3) & 15, c16 = q & 7;
-            const uint4 x = *reinterpret_cast<const uint4 *>(
-                src + vt * L::kKTile + r * 128 + ((c16 ^ (r & 7)) << 4));
-            uint4 lo, hi;
-            lo.x = e4m3x2_to_f16x2(x.x & 0xffffu);
-            lo.y = e4m3x2_to_f16x2(x.x >> 16);
-            lo.z = e4m3x2_to_f16x2(x.y & 0xffffu);
-            lo.w = e4m3x2_to_f16x2(x.y >> 16);
-            hi.x = e4m3x2_to_f16x2(x.z & 0xffffu);
-            hi.y = e4m3x2_to_f16x2(x.z >> 16);
-            hi.z = e4m3x2_to_f16x2(x.w & 0xffffu);
-            hi.w = e4m3x2_to_f16x2(x.w >> 16);
-            uint8_t *t = dst + vt * (kTile * D * 2);
-            *reinterpret_cast<uint4 *>(t + sw128_offset(r, c16 * 16, kTile)) = lo;
-            *reinterpret_cast<uint4 *>(t + sw128_offset(r, c16 * 16 + 8, kTile)) = hi;
-          }
-        }
-        __syncwarp();            // the stage is read: refill it now
-        if (!aborted) issue_next();
-        __syncwarp();            // the widened tiles are written
-        kb = smem_u32(wide);
-      }
+      const uint32_t kb = ring_base + st * L::kStage;
       if (ntok > 0) {
-        const uint32_t vb = kb + (KV8 ? kTile * D * 2 : L::kKTile);
+        const uint32_t vb = kb + L::kKTile;
+        // float8: per-lane row address of the ldmatrix blocks of a 16 x 128-byte
+        // tile (block j = lane / 8: tokens 8 (j & 1) .. +7, 16-byte chunk 2 x + j / 2)
+        const int x8_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+        auto x8_addr = [&](uint32_t tile, int x) {
+          const int c = 2 * x + (lane >> 4);
+          return tile + x8_row * 128 + ((c ^ (x8_row & 7)) << 4);
+        };
         // S^T (16 tokens x 8NT heads) = K Q^T
         float s[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        if (KV8) {
+          // an ldmatrix block of 8 tokens x 16 codes gives lane (g, tq) the codes of
+          // dims 4 tq .. 4 tq + 3 of token g: fragment columns (2tq, 2tq+1) and
+          // (2tq+8, 2tq+9) after widening (the query matches, see load_q)
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t a[4];
-          ldsm_x4(kb + sw128_offset(k_row, ks * 16 + k_col, kTile), a);
+          for (int x = 0; x < KS / 2; ++x) {
+            uint32_t r[4];
+            ldsm_x4(x8_addr(kb, x), r);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_16816<CT>(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+            for (int h = 0; h < 2; ++h) {
+              uint32_t a[4];
+              e4m3x4_to_f16x2(r[2 * h], a[0], a[2]);      // token g
+              e4m3x4_to_f16x2(r[2 * h + 1], a[1], a[3]);  // token g + 8
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma_16816<CT>(s[nt], a, qf[nt][2 * x + h][0], qf[nt][2 * x + h][1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            ldsm_x4(kb + sw128_offset(k_row, ks * 16 + k_col, kTile), a);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_16816<CT>(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+          }
         }
         // online softmax over the tile's tokens (rows g and g + 8 of this lane)
         const bool v0 = g < ntok, v1 = g + 8 < ntok;
@@ -448,23 +447,52 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
         const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
         // O^T (D x 8NT) += V^T P
+        if (KV8) {
+          // a transposed ldmatrix block (8 tokens x 16 codes read as 8 x 8 pairs)
+          // gives lane (g, tq) the codes of dims 16 c + 2g, 16 c + 2g + 1 for tokens
+          // t0 + 2tq, t0 + 2tq + 1; one byte permute pairs them per dim.  So m-tile
+          // c's fragment rows g and g + 8 are dims 16 c + 2g and 16 c + 2g + 1
+          // (the epilogue writes them there).
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          uint32_t a[4];
-          ldsm_x4_trans(vb + sw128_offset(v_row, mt * 16 + v_col, kTile), a);
-          a[0] &= mlo;
-          a[1] &= mlo;
-          a[2] &= mhi;
-          a[3] &= mhi;
+          for (int x = 0; x < KS / 2; ++x) {
+            uint32_t r[4];
+            ldsm_x4_trans(x8_addr(vb, x), r);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
-            mma_16816<CT>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+            for (int h = 0; h < 2; ++h) {
+              const int mt = 2 * x + h;
+              uint32_t a[4];
+              e4m3x4_to_f16x2(__byte_perm(r[2 * h], 0u, 0x3120u), a[0], a[1]);      // tokens 2tq..
+              e4m3x4_to_f16x2(__byte_perm(r[2 * h + 1], 0u, 0x3120u), a[2], a[3]);  // 2tq + 8..
+              a[0] &= mlo;
+              a[1] &= mlo;
+              a[2] &= mhi;
+              a[3] &= mhi;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+                mma_16816<CT>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a[4];
+            ldsm_x4_trans(vb + sw128_offset(v_row, mt * 16 + v_col, kTile), a);
+            a[0] &= mlo;
+            a[1] &= mlo;
+            a[2] &= mhi;
+            a[3] &= mhi;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+              mma_16816<CT>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+            }
           }
         }
       }
       __syncwarp();              // every lane is done with this stage
-      if (!KV8 && !aborted) issue_next();
+      if (!aborted) issue_next();
     }
 
     // ---- finish the segment (or this warp's piece of it)
@@ -492,7 +520,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            const int d = mt * 16 + g + hf * 8;
+            const int d = KV8 ? mt * 16 + 2 * g + hf : mt * 16 + g + hf * 8;
             const float val = o[mt][nt][hf * 2 + e] * inv;
             if (whole) orow[h * D + d] = to16<BF16>(val);
             else p.part_o[(slot * p.G + h) * D + d] = val;

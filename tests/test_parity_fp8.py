@@ -119,3 +119,19 @@ def test_full_size_fp8_sampled(cuda_device):
     hs = torch.randint(0, w.num_q_heads, (48,), generator=g).tolist()
     pairs = np.array(list(zip(bs_, hs)), np.int32)
     assert_close(out[pairs[:, 0], pairs[:, 1]], ref_of(inp, pairs=pairs), "gqa_fp8 full")
+
+
+def test_subnormal_codes_are_exact(cuda_device):
+    # every key / value code subnormal (exponent field 0): with scales 2^7 they
+    # carry values up to 1.75, so any loss of the smallest codes would show
+    inp = workloads.make(kv8(3, 8, 2, 16, (40, 333, 5), seed=11))
+    g = torch.Generator().manual_seed(3)
+    for name in ("k_cache", "v_cache"):
+        c = torch.randint(0, 8, inp[name].shape, generator=g, dtype=torch.int32)
+        sign = torch.randint(0, 2, inp[name].shape, generator=g, dtype=torch.int32) << 7
+        inp[name] = (c | sign).to(torch.uint8)
+    ref = ref_of(inp, k_scale=128.0, v_scale=128.0)
+    d = to_dev(inp, cuda_device)
+    for parts in (0, 5):
+        assert_close(run(d, inp, k_scale=128.0, v_scale=128.0, num_partitions=parts), ref,
+                     f"subnormal parts={parts}")
