@@ -66,8 +66,10 @@ def _load():
             p8 = ctypes.POINTER(ctypes.c_uint8)
             lib.pa_oracle_decode_kv8.argtypes = [i] * 8 + [p16, p8, p8, d, d, p32, p32, d, p32, i,
                                                            pf64, i]
+            lib.pa_oracle_decode_indexed.argtypes = [i] * 8 + [p16, p16, p16, p32, p32, i, p32, d,
+                                                               p32, i, pf64, i]
             for f in (lib.pa_oracle_decode, lib.pa_oracle_decode_split, lib.pa_oracle_decode_mla,
-                      lib.pa_oracle_decode_kv8):
+                      lib.pa_oracle_decode_kv8, lib.pa_oracle_decode_indexed):
                 f.restype = ctypes.c_int
             lib.pa_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
             lib.pa_oracle_f16_to_f64.restype = ctypes.c_double
@@ -183,6 +185,38 @@ def decode_kv8(q, k_cache, v_cache, k_scale, v_scale, block_table, context_lens,
                                   _ptr(bt, ctypes.c_int32), _ptr(cl, ctypes.c_int32), float(scale),
                                   None if pp is None else _ptr(pp, ctypes.c_int32), npairs,
                                   _ptr(out, ctypes.c_double), int(nthreads))
+    _check(rc)
+    return out
+
+
+def decode_indexed(q, k_cache, v_cache, block_table, token_index, n_sel, scale, dtype,
+                   pairs=None, nthreads=0):
+    """Paged GQA decode over a given list of token positions per sequence.
+
+    token_index [B, max_sel] int32 positions (block block_table[b][pos // bs], row
+    pos % bs); n_sel [B] int32 counts.  Other arguments as decode().  Returns
+    float64 [B,Hq,D] (or [len(pairs), D]).
+    """
+    lib = _load()
+    q, k, v = _u16(q), _u16(k_cache), _u16(v_cache)
+    bt, ti, ns = _i32(block_table), _i32(token_index), _i32(n_sel)
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k.shape
+    assert D2 == D and v.shape == k.shape and bt.shape[0] == B and ti.shape[0] == B
+    if pairs is None:
+        out = np.empty((B, Hq, D), np.float64)
+        pp, npairs = None, 0
+    else:
+        pp = _i32(pairs).reshape(-1, 2)
+        npairs = pp.shape[0]
+        out = np.empty((npairs, D), np.float64)
+    rc = lib.pa_oracle_decode_indexed(B, Hq, Hkv, D, bs, bt.shape[1], NB, _dtype_code(dtype),
+                                      _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+                                      _ptr(v, ctypes.c_uint16), _ptr(bt, ctypes.c_int32),
+                                      _ptr(ti, ctypes.c_int32), ti.shape[1],
+                                      _ptr(ns, ctypes.c_int32), float(scale),
+                                      None if pp is None else _ptr(pp, ctypes.c_int32), npairs,
+                                      _ptr(out, ctypes.c_double), int(nthreads))
     _check(rc)
     return out
 

@@ -259,6 +259,69 @@ int pa_oracle_decode_kv8(int B, int Hq, int Hkv, int D, int bs, int mbs, int nb,
 }
 
 /*
+ * Index-list paged decode: each sequence attends over a given list of its token
+ * positions instead of [0, context length) -- the dense kernel behind sparse
+ * attention that keeps only selected entries (page "bjpcjp.github.io:
+ * llms-attention", DeepSeek-V4 explainer: a top-k indexer keeps the top 1024
+ * entries per query, and HCA attends densely over all kept entries).  The
+ * selection itself is an input.
+ *
+ * token_index  [B][max_sel] int32: positions, each < mbs * bs (a position's block
+ *              is block_table[b][pos / bs], row pos % bs); entries past n_sel[b]
+ *              are never read.  A position listed twice counts twice.
+ * n_sel        [B] int32: number of selected positions (0 = all-zero output row).
+ * Everything else as pa_oracle_decode.
+ */
+int pa_oracle_decode_indexed(int B, int Hq, int Hkv, int D, int bs, int mbs, int nb, int dtype,
+                             const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int32_t *block_table, const int32_t *token_index,
+                             int max_sel, const int32_t *n_sel, double scale,
+                             const int32_t *pairs, int npairs, double *out, int nthreads) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0 || mbs < 0 || nb < 0 ||
+      max_sel < 0)
+    return PA_ORACLE_BAD_ARG;
+  const int G = Hq / Hkv;
+  const long n_out = pairs ? (long)npairs : (long)B * Hq;
+  int status = PA_ORACLE_OK;
+#ifdef _OPENMP
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+  for (long i = 0; i < n_out; ++i) {
+    int b = pairs ? pairs[2 * i] : (int)(i / Hq);
+    int h = pairs ? pairs[2 * i + 1] : (int)(i % Hq);
+    double *o = out + i * D;
+    if (b < 0 || b >= B || h < 0 || h >= Hq) { set_status(&status, PA_ORACLE_BAD_ARG); continue; }
+    int n = n_sel[b];
+    if (n < 0 || n > max_sel) { set_status(&status, PA_ORACLE_BAD_ARG); continue; }
+    if (n == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+    int g = h / G;
+    double *qd = malloc(sizeof(double) * D);
+    double *s = malloc(sizeof(double) * n);
+    double *V = malloc(sizeof(double) * (size_t)n * D);
+    if (!qd || !s || !V) { free(qd); free(s); free(V); set_status(&status, PA_ORACLE_NO_MEMORY); continue; }
+    for (int d = 0; d < D; ++d) qd[d] = decode16(q[((long)b * Hq + h) * D + d], dtype);
+    int bad = 0;
+    for (int t = 0; t < n; ++t) {
+      int pos = token_index[(long)b * max_sel + t];
+      long blk = pos < 0 ? -1 : block_of(block_table, mbs, nb, bs, b, pos);
+      if (blk < 0) { bad = 1; break; }
+      long row = ((blk * Hkv + g) * bs + pos % bs) * (long)D;
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) {
+        acc += qd[d] * decode16(k_cache[row + d], dtype);
+        V[(long)t * D + d] = decode16(v_cache[row + d], dtype);
+      }
+      s[t] = scale * acc;
+    }
+    if (bad) set_status(&status, PA_ORACLE_BAD_BLOCK);
+    else softmax_mix(n, s, V, D, o);
+    free(qd); free(s); free(V);
+  }
+  return status;
+}
+
+/*
  * The same GQA operation computed the Flash-Decoding way, as an independent
  * statement for the split-then-merge property: tokens [0, n) are cut into splits
  * of split_len tokens; each split yields o_s (normalised) and

@@ -328,3 +328,67 @@ def test_kv8_value_scale_scales_the_output():
     a = _run_kv8(inp, v_scale=0.37)
     b = _run_kv8(inp, v_scale=1.0) * 0.37
     np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- index-list decode
+
+def _indexed_small(seed=0, ctx=200, top=20, window=8):
+    w = workloads.IndexedWorkload("t", 3, 4, 2, 16, "bf16", 8, ctx, top, window, seed)
+    return workloads.make_indexed(w)
+
+
+def _run_indexed(inp, token_index=None, n_sel=None):
+    return oracle.decode_indexed(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
+                                 inp["block_table"].numpy(),
+                                 (inp["token_index"] if token_index is None else token_index).numpy(),
+                                 (inp["n_sel"] if n_sel is None else n_sel).numpy(),
+                                 inp["scale"], inp["dtype"])
+
+
+def test_indexed_decode_equals_dense_decode_of_the_gathered_rows():
+    # brute force: copy the selected rows, in list order, into a fresh contiguous
+    # paged cache and run the (pinned) dense definition over it
+    inp = _indexed_small()
+    B, bs = inp["q"].shape[0], 8
+    k, v, bt, sel = inp["k_cache"], inp["v_cache"], inp["block_table"], inp["token_index"]
+    n = sel.shape[1]
+    nblk = (n + bs - 1) // bs
+    kd = torch.zeros((B * nblk, k.shape[1], bs, k.shape[3]), dtype=k.dtype)
+    vd = torch.zeros_like(kd)
+    for b in range(B):
+        for i, pos in enumerate(sel[b].tolist()):
+            phys = int(bt[b, pos // bs])
+            kd[b * nblk + i // bs, :, i % bs] = k[phys, :, pos % bs]
+            vd[b * nblk + i // bs, :, i % bs] = v[phys, :, pos % bs]
+    table = torch.arange(B * nblk, dtype=torch.int32).view(B, nblk)
+    ref = oracle.decode(u16(inp["q"]), u16(kd), u16(vd), table.numpy(),
+                        inp["n_sel"].numpy(), inp["scale"], inp["dtype"])
+    assert np.array_equal(_run_indexed(inp), ref)
+
+
+def test_indexed_decode_with_every_position_equals_dense_decode():
+    inp = _indexed_small(seed=1, ctx=48, top=0, window=48)   # the whole context, in order
+    ref = oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
+                        inp["block_table"].numpy(), inp["context_lens"].numpy(), inp["scale"],
+                        inp["dtype"])
+    assert np.array_equal(_run_indexed(inp), ref)
+
+
+def test_indexed_decode_ignores_the_order_of_the_list():
+    inp = _indexed_small(seed=2)
+    g = torch.Generator().manual_seed(5)
+    shuffled = torch.stack([r[torch.randperm(r.numel(), generator=g)] for r in inp["token_index"]])
+    np.testing.assert_allclose(_run_indexed(inp, token_index=shuffled), _run_indexed(inp),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_indexed_decode_reads_only_the_first_n_sel_entries():
+    inp = _indexed_small(seed=3)
+    ns = torch.tensor([5, 0, 28], dtype=torch.int32)
+    poisoned = inp["token_index"].clone()
+    poisoned[0, 5:] = -7
+    poisoned[1, :] = 10 ** 6
+    a = _run_indexed(inp, token_index=poisoned, n_sel=ns)
+    b = _run_indexed(inp, n_sel=ns)
+    assert np.array_equal(a, b)
+    assert np.all(a[1] == 0)

@@ -217,11 +217,77 @@ def make(w, context_lens: Optional[torch.Tensor] = None):
                 max_blocks_per_seq=mbs)
 
 
+@dataclass(frozen=True)
+class IndexedWorkload:
+    """GQA decode over a per-sequence list of selected token positions."""
+    name: str
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    dtype: str
+    block_size: int
+    ctx: int              # context length of every sequence
+    top: int              # positions drawn uniformly from [0, ctx - window)
+    window: int           # plus the last `window` positions
+    seed: int
+
+    @property
+    def kind(self):
+        return "gqa_indexed"
+
+    @property
+    def n_sel(self):
+        return self.top + self.window
+
+
+# Index-list decode (the dense kernel behind sparse top-k attention; the pages'
+# DeepSeek-V4 explainer: keep the top 1024 entries plus a 128-token sliding
+# window).  The selection is an input: 1024 positions drawn uniformly without
+# replacement from [0, ctx - 128), sorted, plus the last 128.  Only blocks that
+# hold a selected token are in the pool; every other table entry is -1.
+INDEXED = {
+    "topk": IndexedWorkload("topk", 32, 32, 8, 128, "bf16", 16, 32768, 1024, 128, 1008),
+}
+
+
+def make_indexed(w: IndexedWorkload, n_sel: Optional[torch.Tensor] = None):
+    """Draw the inputs of an index-list workload on the CPU (optionally with fewer
+    selected positions per sequence, n_sel[b] <= w.n_sel, keeping the first ones)."""
+    gen = torch.Generator().manual_seed(w.seed)
+    B, bs = w.batch, w.block_size
+    mbs = (w.ctx + bs - 1) // bs
+    sel = torch.empty((B, w.n_sel), dtype=torch.int32)
+    for b in range(B):
+        top = torch.randperm(w.ctx - w.window, generator=gen)[:w.top].sort().values
+        win = torch.arange(w.ctx - w.window, w.ctx)
+        sel[b] = torch.cat([top, win]).to(torch.int32)
+    used = [sorted(set((sel[b] // bs).tolist())) for b in range(B)]
+    nb = sum(len(u) for u in used)
+    perm = torch.randperm(nb, generator=gen).to(torch.int32)
+    table = torch.full((B, mbs), -1, dtype=torch.int32)
+    k = 0
+    for b in range(B):
+        for lb in used[b]:
+            table[b, lb] = perm[k]
+            k += 1
+    q = _randn16((B, w.num_q_heads, w.head_dim), w.dtype, gen)
+    kv_shape = (nb, w.num_kv_heads, bs, w.head_dim)
+    kc, vc = _randn16(kv_shape, w.dtype, gen), _randn16(kv_shape, w.dtype, gen)
+    ns = torch.full((B,), w.n_sel, dtype=torch.int32) if n_sel is None else n_sel.to(torch.int32)
+    return dict(kind="gqa_indexed", q=q, k_cache=kc, v_cache=vc, block_table=table,
+                token_index=sel, n_sel=ns, context_lens=torch.full((B,), w.ctx, dtype=torch.int32),
+                scale=1.0 / math.sqrt(w.head_dim), dtype=w.dtype, num_blocks=nb,
+                max_blocks_per_seq=mbs)
+
+
 def kv_bytes(w, context_lens: torch.Tensor) -> int:
     """Bytes of live KV the operation must read once: every cached element of
     every live token (q, out, block table and scratch excluded).  MLA counts the
     latent once because the value is a prefix of it."""
     tokens = int(context_lens.to(torch.int64).sum())
+    if w.kind == "gqa_indexed":        # context_lens here: the selected counts n_sel
+        return tokens * w.num_kv_heads * w.head_dim * 2 * 2
     if w.kind == "gqa":
         elem = 1 if w.kv_dtype == "e4m3" else 2
         return tokens * w.num_kv_heads * w.head_dim * 2 * elem
