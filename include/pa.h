@@ -164,11 +164,32 @@ pa_status pa_decode_kv_e4m3(const pa_desc *desc, const void *q, const void *k_ca
                             float v_scale, void *out, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/* Index-list decode: each sequence attends over a given list of its token
+ * positions instead of [0, context length), the dense kernel behind sparse
+ * attention that keeps selected entries (page "bjpcjp.github.io: llms-attention",
+ * DeepSeek-V4 explainer: keep the top 1024 entries plus a sliding window, then
+ * attend over them).  The selection is an input.
+ *
+ * token_index: device int32 [batch][max_sel]; entry i < n_sel[b] is a token
+ *   position of sequence b (its K/V row is row pos % block_size of block
+ *   block_table[b][pos / block_size]); entries past n_sel[b] are never read, a
+ *   position listed twice counts twice, the order does not matter.
+ * n_sel: device int32 [batch], 0 <= n_sel[b] <= max_sel (0 = all-zero output).
+ * Everything else as pa_decode (16-bit q / caches / out, head_dim 128).  A
+ * position outside [0, max_blocks_per_seq x block_size) or a block id outside
+ * the pool is skipped and reported as PA_ERR_BAD_BLOCK_ID by pa_device_status.
+ * The workspace is sized by pa_workspace_size(desc). */
+pa_status pa_decode_indexed(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *token_index, int max_sel, const int32_t *n_sel,
+                            float scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
 /* Number of partitions (CTAs of the partition pass; each runs 8 independently
  * streaming warps, one piece each) a call with num_partitions == 0 uses on the current
  * device (SM count x resident CTAs per SM), or -1 without a usable device.
  * kind: 0 = GQA with this head_dim, 1 = MLA (head_dim ignored), 2 = GQA over a
- * float8 KV cache (head_dim 128). */
+ * float8 KV cache (head_dim 128), 3 = index-list decode (head_dim 128). */
 int pa_default_partitions(int kind, int head_dim);
 
 /* Synchronises `stream`, then returns the first error the kernels recorded on the

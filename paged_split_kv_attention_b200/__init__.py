@@ -77,6 +77,9 @@ def library() -> ctypes.CDLL:
             lib.pa_decode_kv_e4m3.argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp, f32, f32,
                                               f32, vp, vp, sz, vp]
             lib.pa_decode_kv_e4m3.restype = ctypes.c_int
+            lib.pa_decode_indexed.argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp,
+                                              ctypes.c_int, vp, f32, vp, vp, sz, vp]
+            lib.pa_decode_indexed.restype = ctypes.c_int
             lib.pa_workspace_size.argtypes = [ctypes.POINTER(PADesc)]
             lib.pa_workspace_size.restype = sz
             lib.pa_mla_workspace_size.argtypes = [ctypes.POINTER(PAMLADesc)]
@@ -141,8 +144,8 @@ def workspace_size(desc) -> int:
 
 
 def default_partitions(kind: str = "gqa", head_dim: int = 128) -> int:
-    """kind: "gqa", "mla" or "gqa_fp8" (GQA over a float8 KV cache)."""
-    code = {"gqa": 0, "mla": 1, "gqa_fp8": 2}[kind]
+    """kind: "gqa", "mla", "gqa_fp8" (float8 KV cache) or "gqa_indexed" (index list)."""
+    code = {"gqa": 0, "mla": 1, "gqa_fp8": 2, "gqa_indexed": 3}[kind]
     return int(library().pa_default_partitions(code, head_dim))
 
 
@@ -242,6 +245,38 @@ def decode_kv8(q, k_cache, v_cache, block_table, context_lens, scale, k_scale, v
                                        float(k_scale), float(v_scale), _ptr(out), _ptr(ws),
                                        ws.numel() * ws.element_size(), _stream_ptr(stream)),
            "pa_decode_kv_e4m3")
+    return out
+
+
+def decode_indexed(q, k_cache, v_cache, block_table, token_index, n_sel, scale, out=None,
+                   workspace=None, num_partitions=0, stream=None):
+    """pa_decode_indexed: each sequence attends over a list of its token positions.
+
+    token_index [B, max_sel] int32 positions; n_sel [B] int32 counts (entries past
+    n_sel[b] are never read).  Caches and q as decode() (head_dim 128).
+    """
+    _require(q, "q", ndim=3)
+    _require(k_cache, "k_cache", q.dtype, 4)
+    _require(v_cache, "v_cache", q.dtype, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(token_index, "token_index", torch.int32, 2)
+    _require(n_sel, "n_sel", torch.int32, 1)
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache shapes differ")
+    desc = gqa_desc(q, k_cache, block_table, num_partitions)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _require(out, "out", q.dtype, 3)
+    ws_bytes = workspace_size(desc)
+    if ws_bytes == 0:
+        raise PAError(PA_ERR_UNSUPPORTED, "pa_workspace_size")
+    ws = _workspace(ws_bytes, q.device, workspace)
+    _check(library().pa_decode_indexed(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(block_table), _ptr(token_index),
+                                       int(token_index.shape[1]), _ptr(n_sel), float(scale),
+                                       _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream_ptr(stream)), "pa_decode_indexed")
     return out
 
 

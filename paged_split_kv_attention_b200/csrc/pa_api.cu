@@ -97,41 +97,45 @@ int resident_ctas(const void *kernel, int threads, size_t smem) {
 
 // ------------------------------------------------------------------ GQA variants
 
-template <int D, int NT, bool BF16, bool KV8>
+// Kernel modes: 16-bit cache, float8 cache, index-list decode.
+enum GqaMode { kMode16 = 0, kModeKv8 = 1, kModeIndexed = 2 };
+
+template <int D, int NT, bool BF16, int MODE>
 struct GqaVariant {
   // 24 KB ring per warp: 3 x 8 KB (D 128), 6 x 4 KB (D 64 or float8 D 128)
-  static constexpr int R = KV8 ? 6 : (D == 128 ? 3 : 6);
-  using L = pa::GqaLayout<D, NT, R, KV8>;
+  static constexpr int R = MODE == kModeKv8 ? 6 : (D == 128 ? 3 : 6);
+  using L = pa::GqaLayout<D, NT, R, MODE == kModeKv8>;
   static const void *kernel() {
-    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, KV8>);
+    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, MODE>);
   }
   static void launch(int grid, size_t smem, cudaStream_t st, const CUtensorMap &k,
                      const CUtensorMap &v, const pa::GqaParams &p) {
-    pa::gqa_decode_kernel<D, NT, BF16, R, KV8><<<grid, pa::kGqaThreads, smem, st>>>(k, v, p);
+    pa::gqa_decode_kernel<D, NT, BF16, R, MODE><<<grid, pa::kGqaThreads, smem, st>>>(k, v, p);
   }
 };
 
-template <template <int, int, bool, bool> class F, typename... A>
-bool dispatch_gqa(int D, int NT, bool bf16, bool kv8, A &&...a) {
-#define PA_CASE(d, nt, b, k8)                               \
-  if (D == d && NT == nt && bf16 == b && kv8 == k8) {       \
-    F<d, nt, b, k8>::run(static_cast<A &&>(a)...);          \
+template <template <int, int, bool, int> class F, typename... A>
+bool dispatch_gqa(int D, int NT, bool bf16, int mode, A &&...a) {
+#define PA_CASE(d, nt, b, m)                                \
+  if (D == d && NT == nt && bf16 == b && mode == m) {       \
+    F<d, nt, b, m>::run(static_cast<A &&>(a)...);           \
     return true;                                            \
   }
-  PA_CASE(128, 1, true, false) PA_CASE(128, 1, false, false)
-  PA_CASE(128, 2, true, false) PA_CASE(128, 2, false, false)
-  PA_CASE(64, 1, true, false) PA_CASE(64, 1, false, false)
-  PA_CASE(64, 2, true, false) PA_CASE(64, 2, false, false)
-  PA_CASE(128, 1, true, true) PA_CASE(128, 1, false, true)
-  PA_CASE(128, 2, true, true) PA_CASE(128, 2, false, true)
+  PA_CASE(128, 1, true, 0) PA_CASE(128, 1, false, 0) PA_CASE(128, 2, true, 0)
+  PA_CASE(128, 2, false, 0) PA_CASE(64, 1, true, 0) PA_CASE(64, 1, false, 0)
+  PA_CASE(64, 2, true, 0) PA_CASE(64, 2, false, 0)
+  PA_CASE(128, 1, true, 1) PA_CASE(128, 1, false, 1) PA_CASE(128, 2, true, 1)
+  PA_CASE(128, 2, false, 1)
+  PA_CASE(128, 1, true, 2) PA_CASE(128, 1, false, 2) PA_CASE(128, 2, true, 2)
+  PA_CASE(128, 2, false, 2)
 #undef PA_CASE
   return false;
 }
 
-template <int D, int NT, bool BF16, bool KV8>
+template <int D, int NT, bool BF16, int MODE>
 struct QueryResident {
   static void run(int B, int *out) {
-    using V = GqaVariant<D, NT, BF16, KV8>;
+    using V = GqaVariant<D, NT, BF16, MODE>;
     *out = resident_ctas(V::kernel(), pa::kGqaThreads, V::L::bytes(B));
   }
 };
@@ -141,15 +145,15 @@ struct GqaPlan {
   size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
-int default_gqa_parts(int D, int NT, bool bf16, bool kv8, int B) {
+int default_gqa_parts(int D, int NT, bool bf16, int mode, int B) {
   const int sms = sm_count();
   if (sms <= 0) return -1;
   int per = -1;
-  if (!dispatch_gqa<QueryResident>(D, NT, bf16, kv8, B, &per) || per <= 0) return -1;
+  if (!dispatch_gqa<QueryResident>(D, NT, bf16, mode, B, &per) || per <= 0) return -1;
   return sms * per;
 }
 
-pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, bool kv8 = false) {
+pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, int mode = kMode16) {
   if (!d) return PA_ERR_INVALID_ARG;
   if (d->batch < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0 ||
       d->block_size <= 0 || d->max_blocks_per_seq <= 0 || d->num_blocks <= 0 ||
@@ -160,7 +164,7 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, bool kv8 = false) {
   const int G = d->num_q_heads / d->num_kv_heads;
   if (G > 16) return PA_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (kv8 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (mode != kMode16 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (d->block_size % pa::kTile || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
   if (d->batch > kMaxBatch) return PA_ERR_UNSUPPORTED;
   const int64_t kv_rows = int64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
@@ -173,7 +177,7 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, bool kv8 = false) {
   pl->NT = G <= 8 ? 1 : 2;
   pl->parts = d->num_partitions;
   if (pl->parts == 0) {
-    pl->parts = default_gqa_parts(d->head_dim, pl->NT, d->dtype == PA_BF16, kv8, d->batch);
+    pl->parts = default_gqa_parts(d->head_dim, pl->NT, d->dtype == PA_BF16, mode, d->batch);
     if (pl->parts <= 0) return PA_ERR_CUDA;
   }
   // one partial slot per (warp piece, segment) pair a piece can end: piece + segment
@@ -199,11 +203,11 @@ pa_status check_gqa_args(const pa_desc *d, const GqaPlan &pl, const void *q, con
   return PA_OK;
 }
 
-template <int D, int NT, bool BF16, bool KV8>
+template <int D, int NT, bool BF16, int MODE>
 struct LaunchPartition {
   static void run(int grid, cudaStream_t st, const CUtensorMap *maps, const pa::GqaParams *p,
                   cudaError_t *err) {
-    using V = GqaVariant<D, NT, BF16, KV8>;
+    using V = GqaVariant<D, NT, BF16, MODE>;
     const size_t smem = V::L::bytes(p->B);
     *err = cudaFuncSetAttribute(V::kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(smem));
@@ -288,18 +292,24 @@ std::atomic<int> g_stall_test{0};
 
 enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
 
-// kv8: k / v hold float8 E4M3 codes, key = code x k_scale, value = code x v_scale.
+// mode kModeKv8: k / v hold float8 E4M3 codes, key = code x k_scale, value =
+// code x v_scale.  kModeIndexed: cl holds the selected counts and token_index
+// [B][max_sel] the selected positions.
 pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, const void *v,
                   const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
-                  size_t ws_bytes, void *stream, bool kv8 = false, float k_scale = 1.f,
-                  float v_scale = 1.f) {
+                  size_t ws_bytes, void *stream, int mode = kMode16, float k_scale = 1.f,
+                  float v_scale = 1.f, const int32_t *token_index = nullptr, int max_sel = 0) {
+  const bool kv8 = mode == kModeKv8;
   GqaPlan pl;
-  pa_status s = plan_gqa(d, &pl, kv8);
+  pa_status s = plan_gqa(d, &pl, mode);
   if (s != PA_OK) return s;
   if (d->batch == 0) return PA_OK;
   s = check_gqa_args(d, pl, q, k, v, bt, cl, out, ws, ws_bytes);
   if (s != PA_OK) return s;
   if (!std::isfinite(scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return PA_ERR_INVALID_ARG;
+  if (mode == kModeIndexed &&
+      (!token_index || (reinterpret_cast<uintptr_t>(token_index) & 3u) || max_sel <= 0))
     return PA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
@@ -334,10 +344,14 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.parts = pl.parts;
     p.scale_log2 = scale * k_scale * kLog2e;
     p.v_scale = v_scale;
+    p.token_index = token_index;
+    p.max_sel = max_sel;
+    p.k_cache = k;
+    p.v_cache = v;
     p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     p.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
     cudaError_t err = cudaSuccess;
-    if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, kv8, pl.parts, st, maps, &p, &err))
+    if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, mode, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
     if (err != cudaSuccess) return PA_ERR_CUDA;
   }
@@ -487,9 +501,12 @@ size_t pa_workspace_size(const pa_desc *desc) {
   GqaPlan pl;
   if (plan_gqa(desc, &pl) != PA_OK) return 0;
   size_t bytes = pl.bytes;
-  GqaPlan pl8;                       // the float8 KV call may launch another grid size
-  if (desc->head_dim == 128 && plan_gqa(desc, &pl8, true) == PA_OK && pl8.bytes > bytes)
-    bytes = pl8.bytes;
+  // the float8 and index-list calls may launch another grid size
+  for (int mode : {kModeKv8, kModeIndexed}) {
+    GqaPlan other;
+    if (desc->head_dim == 128 && plan_gqa(desc, &other, mode) == PA_OK && other.bytes > bytes)
+      bytes = other.bytes;
+  }
   return bytes;
 }
 
@@ -499,7 +516,16 @@ pa_status pa_decode_kv_e4m3(const pa_desc *desc, const void *q, const void *k_ca
                             float v_scale, void *out, void *workspace, size_t workspace_bytes,
                             void *stream) {
   return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
-                 workspace, workspace_bytes, stream, true, k_scale, v_scale);
+                 workspace, workspace_bytes, stream, kModeKv8, k_scale, v_scale);
+}
+
+pa_status pa_decode_indexed(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *token_index, int max_sel, const int32_t *n_sel,
+                            float scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, n_sel, scale, out, workspace,
+                 workspace_bytes, stream, kModeIndexed, 1.f, 1.f, token_index, max_sel);
 }
 
 pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache, const void *v_cache,
@@ -557,9 +583,10 @@ pa_status pa_decode_mla_merge(const pa_mla_desc *desc, const void *q, const void
 int pa_default_partitions(int kind, int head_dim) {
   if (kind == 0) {
     if (head_dim != 64 && head_dim != 128) return -1;
-    return default_gqa_parts(head_dim, 1, true, false, 256);
+    return default_gqa_parts(head_dim, 1, true, kMode16, 256);
   }
-  if (kind == 2) return head_dim == 128 ? default_gqa_parts(128, 1, true, true, 256) : -1;
+  if (kind == 2) return head_dim == 128 ? default_gqa_parts(128, 1, true, kModeKv8, 256) : -1;
+  if (kind == 3) return head_dim == 128 ? default_gqa_parts(128, 1, true, kModeIndexed, 256) : -1;
   return default_mla_parts();
 }
 

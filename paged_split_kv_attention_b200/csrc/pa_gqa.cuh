@@ -74,6 +74,10 @@ struct GqaParams {
   int stall_test;               // test hook: warp 0 of CTA 0 waits on a barrier nothing completes
   int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
   float v_scale;                // value scale of a float8 KV cache (1 otherwise)
+  // index-list decode (MODE 2): context_lens holds the selected counts n_sel
+  const int32_t *token_index;   // [B][max_sel] token positions
+  int max_sel;
+  const void *k_cache, *v_cache;  // the gathers read the caches directly
 };
 
 template <int D, int NT, int R, bool KV8 = false>
@@ -152,6 +156,24 @@ __device__ __forceinline__ int tile_row(const GqaParams &p, const int *prefix, l
   return (blk * p.Hkv + kvh) * p.bs + (j - jb * p.tiles_per_block) * kTile;
 }
 
+// Index-list decode: cache row of selected entry r of flattened tile t (entry
+// 16 j + r of its sequence's list), -2 past the sequence's selection, -1 for a
+// position outside the table or a block id outside the pool (recorded, never
+// dereferenced).
+__device__ __forceinline__ int indexed_row(const GqaParams &p, const int *prefix, long long t,
+                                           int r) {
+  int b, kvh, j;
+  locate_tile(prefix, p.B, p.Hkv, t, b, kvh, j);
+  const int i = j * kTile + r;
+  const int n = clamp_ctx(__ldg(&p.context_lens[b]), p.max_sel);
+  if (i >= n) return -2;
+  const int pos = __ldg(&p.token_index[static_cast<long long>(b) * p.max_sel + i]);
+  if (pos < 0 || pos >= p.mbs * p.bs) return -1;
+  const int blk = __ldg(&p.block_table[static_cast<long long>(b) * p.mbs + pos / p.bs]);
+  if (blk < 0 || blk >= p.nb) return -1;
+  return (blk * p.Hkv + kvh) * p.bs + pos % p.bs;
+}
+
 // Query B-operand fragments (Q^T: d x heads) of group (b, kvh): for n-tile nt and
 // k-step ks, lane holds Q[head 8nt+g][16ks+2tq .. +1] and Q[..][16ks+8+2tq .. +1];
 // heads past the group are zero.
@@ -197,10 +219,13 @@ __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int l
   }
 }
 
-template <int D, int NT, bool BF16, int R, bool KV8 = false>
+// MODE 0: 16-bit cache, TMA tiles.  1: float8 cache (KV8).  2: index-list
+// decode (IDX): each warp gathers its tiles' selected rows with cp.async.
+template <int D, int NT, bool BF16, int R, int MODE = 0>
 __global__ void __launch_bounds__(kGqaThreads, 1)
 gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
+  constexpr bool KV8 = MODE == 1, IDX = MODE == 2;
   using L = GqaLayout<D, NT, R, KV8>;
   static_assert(!KV8 || D == 128, "the float8 KV path reads 128-byte rows");
   constexpr bool CT = BF16 && !KV8;          // MMA operand type: bf16, else fp16
@@ -215,7 +240,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
-  const int cap = p.mbs * p.bs;
+  const int cap = IDX ? p.max_sel : p.mbs * p.bs;
 
   // Warm L2 with this CTA's share of the block table while the lengths load.
   {
@@ -247,7 +272,8 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   int *stage_valid = reinterpret_cast<int *>(sm + L::info) + warp * R;
   uint8_t *ring = sm + L::ring + warp * R * L::kStage;
   if (lane == 0) {
-    for (int s = 0; s < R; ++s) mbar_init(&full[s], 1);
+    // IDX: 32 lanes' cp.async arrivals + lane 0's arrive after writing stage_valid
+    for (int s = 0; s < R; ++s) mbar_init(&full[s], IDX ? 33 : 1);
     if (warp == 0) *abort_flag = 0;
     fence_barrier_init();
   }
@@ -263,21 +289,54 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 
   const uint64_t policy = l2_evict_first_policy();
-  if (lane == 0) {
+  if (lane == 0 && !IDX) {
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
   }
 
   // ---- look-ahead: lane i holds the cache row of tile la_base + i
+  // (IDX: lane l holds the row of selected entry l % 16 of the next tile to issue)
   long long la_base = wb;
-  int la_row = (wb + lane < we) ? tile_row(p, prefix, wb + lane) : 0;
+  int la_row = (!IDX && wb + lane < we) ? tile_row(p, prefix, wb + lane) : 0;
   long long nx_base = wb + 32;
-  int nx_row = (nx_base + lane < we) ? tile_row(p, prefix, nx_base + lane) : 0;
+  int nx_row = (!IDX && nx_base + lane < we) ? tile_row(p, prefix, nx_base + lane) : 0;
+  int idx_row = (IDX && wb < we) ? indexed_row(p, prefix, wb, lane & 15) : -2;
   long long issued = wb;                              // next tile to issue
 
   // Issue tile `issued` into its stage (lane 0 does the copy; all lanes call).
   auto issue_next = [&]() {
     if (issued >= we) return;
+    if (IDX) {
+      // gather: lane l copies half of selected row l % 16 (K and V), 16 bytes per
+      // cp.async, into the swizzled layout the TMA path produces
+      const long long n = issued - wb;
+      const int st = static_cast<int>(n % R);
+      const bool bad = __any_sync(0xffffffffu, idx_row == -1);
+      if (!bad && idx_row >= 0) {
+        constexpr int kChunks = D / 8;                // 16-byte chunks per row
+        const int r = lane & 15, half = lane >> 4;
+        const char *ks = static_cast<const char *>(p.k_cache) + static_cast<long long>(idx_row) * D * 2;
+        const char *vs = static_cast<const char *>(p.v_cache) + static_cast<long long>(idx_row) * D * 2;
+        const uint32_t dk = smem_u32(ring + st * L::kStage), dv = dk + L::kKTile;
+#pragma unroll
+        for (int cc = 0; cc < kChunks / 2; ++cc) {
+          const int ch = half * (kChunks / 2) + cc;
+          const uint32_t off = sw128_offset(r, ch * 8, kTile);
+          cp_async16(dk + off, ks + ch * 16);
+          cp_async16(dv + off, vs + ch * 16);
+        }
+      }
+      cp_async_mbar_arrive_noinc(&full[st]);
+      if (lane == 0) {
+        if (bad) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
+        stage_valid[st] = bad ? 0 : 1;
+        mbar_arrive(&full[st]);
+      }
+      ++issued;
+      // the next tile's lookups now, so that their latency hides behind this tile
+      idx_row = issued < we ? indexed_row(p, prefix, issued, lane & 15) : -2;
+      return;
+    }
     if (issued >= la_base + 32) {                     // slide the look-ahead window
       la_base = nx_base;
       la_row = nx_row;
@@ -325,6 +384,8 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   locate_tile(prefix, p.B, p.Hkv, wb, b, kvh, j0);
   uint32_t qf[NT][KS][2], nq[NT][KS][2];
   load_q<D, NT, BF16 && KV8, KV8>(p, b, kvh, lane, qf);
+  (void)tm_k;
+  (void)tm_v;
   int ctx = clamp_ctx(__ldg(&p.context_lens[b]), cap);
   bool aborted = false;
 
