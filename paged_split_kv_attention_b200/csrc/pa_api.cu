@@ -104,7 +104,7 @@ template <int D, int NT, bool BF16, int MODE>
 struct GqaVariant {
   // 24 KB ring per warp: 3 x 8 KB (D 128), 6 x 4 KB (D 64 or float8 D 128)
   static constexpr int R = MODE == kModeKv8 ? 6 : (D == 128 ? 3 : 6);
-  using L = pa::GqaLayout<D, NT, R, MODE == kModeKv8>;
+  using L = pa::GqaLayout<D, NT, R, MODE>;
   static const void *kernel() {
     return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, MODE>);
   }

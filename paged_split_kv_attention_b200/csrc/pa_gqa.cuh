@@ -80,10 +80,12 @@ struct GqaParams {
   const void *k_cache, *v_cache;  // the gathers read the caches directly
 };
 
-template <int D, int NT, int R, bool KV8 = false>
+// MODE 0 and 2: 16-bit rows in 128-byte swizzled slabs (2: gathered row by row
+// into the same layout).  MODE 1: float8 rows.
+template <int D, int NT, int R, int MODE = 0>
 struct GqaLayout {
   static constexpr int kHeads = 8 * NT;            // group width padded to the MMA N
-  static constexpr int kKTile = kTile * D * (KV8 ? 1 : 2);  // bytes of one K (or V) tile
+  static constexpr int kKTile = kTile * D * (MODE == 1 ? 1 : 2);  // bytes of one K (or V) tile
   static constexpr int kStage = 2 * kKTile;
   static constexpr int ring = 0;                   // warp w: stages [w*R, (w+1)*R)
   static constexpr int bars = ring + kWarps * R * kStage;
@@ -156,22 +158,48 @@ __device__ __forceinline__ int tile_row(const GqaParams &p, const int *prefix, l
   return (blk * p.Hkv + kvh) * p.bs + (j - jb * p.tiles_per_block) * kTile;
 }
 
-// Index-list decode: cache row of selected entry r of flattened tile t (entry
-// 16 j + r of its sequence's list), -2 past the sequence's selection, -1 for a
-// position outside the table or a block id outside the pool (recorded, never
-// dereferenced).
-__device__ __forceinline__ int indexed_row(const GqaParams &p, const int *prefix, long long t,
-                                           int r) {
-  int b, kvh, j;
-  locate_tile(prefix, p.B, p.Hkv, t, b, kvh, j);
-  const int i = j * kTile + r;
-  const int n = clamp_ctx(__ldg(&p.context_lens[b]), p.max_sel);
-  if (i >= n) return -2;
-  const int pos = __ldg(&p.token_index[static_cast<long long>(b) * p.max_sel + i]);
-  if (pos < 0 || pos >= p.mbs * p.bs) return -1;
-  const int blk = __ldg(&p.block_table[static_cast<long long>(b) * p.mbs + pos / p.bs]);
-  if (blk < 0 || blk >= p.nb) return -1;
-  return (blk * p.Hkv + kvh) * p.bs + pos % p.bs;
+// Index-list decode: the lookups behind selected entry r (= lane % 16) of a
+// tile form a three-step chain of dependent loads (count -> position -> block
+// id).  Each step runs one tile apart, at successive issues, so every load has a
+// tile's worth of time to land and no lane waits on one.
+struct IdxLookup {
+  int b3 = 0, kvh3 = 0, j3 = 0, n3 = 0, live3 = 0;   // located; count loading
+  int b2 = 0, kvh2 = 0, pos2 = -2;                  // position loading (-2: none)
+  int kvh1 = 0, pos1 = -2, blk1 = -1;               // block id loading (-1: bad)
+};
+
+// Advance the chain by one tile: the located tile moves on to its position load,
+// the position to its block-id load, and tile t enters (live if t < end).
+__device__ __forceinline__ void idx_advance(const GqaParams &p, const int *prefix, IdxLookup &k,
+                                            long long t, long long end, int r) {
+  k.kvh1 = k.kvh2;
+  k.pos1 = k.pos2;
+  if (k.pos2 >= 0 && k.pos2 < p.mbs * p.bs) {
+    k.blk1 = __ldg(&p.block_table[static_cast<long long>(k.b2) * p.mbs + k.pos2 / p.bs]);
+  } else {
+    k.blk1 = -1;
+    if (k.pos2 != -2) k.pos1 = -1;                  // a position outside the table
+  }
+  k.b2 = k.b3;
+  k.kvh2 = k.kvh3;
+  const int i = k.j3 * kTile + r;
+  k.pos2 = (k.live3 && i < k.n3)
+               ? __ldg(&p.token_index[static_cast<long long>(k.b3) * p.max_sel + i]) : -2;
+  if (k.pos2 < 0 && k.pos2 != -2) k.pos2 = -1;
+  k.live3 = t < end;
+  if (k.live3) {
+    locate_tile(prefix, p.B, p.Hkv, t, k.b3, k.kvh3, k.j3);
+    k.n3 = __ldg(&p.context_lens[k.b3]);            // the selected count
+    k.n3 = k.n3 < 0 ? 0 : (k.n3 > p.max_sel ? p.max_sel : k.n3);
+  }
+}
+
+// Cache row of the tile at the end of the chain: -2 no entry, -1 bad (recorded
+// by the caller, never dereferenced).
+__device__ __forceinline__ int idx_row_of(const GqaParams &p, const IdxLookup &k) {
+  if (k.pos1 == -2) return -2;
+  if (k.pos1 < 0 || k.blk1 < 0 || k.blk1 >= p.nb) return -1;
+  return (k.blk1 * p.Hkv + k.kvh1) * p.bs + k.pos1 % p.bs;
 }
 
 // Query B-operand fragments (Q^T: d x heads) of group (b, kvh): for n-tile nt and
@@ -226,8 +254,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
 gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
   constexpr bool KV8 = MODE == 1, IDX = MODE == 2;
-  using L = GqaLayout<D, NT, R, KV8>;
+  using L = GqaLayout<D, NT, R, MODE>;
   static_assert(!KV8 || D == 128, "the float8 KV path reads 128-byte rows");
+  static_assert(!IDX || D == 128, "index-list gathers read 256-byte rows");
   constexpr bool CT = BF16 && !KV8;          // MMA operand type: bf16, else fp16
   constexpr int KS = D / 16;                 // k-steps of the score MMA / m-tiles of the PV MMA
 
@@ -300,30 +329,37 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   int la_row = (!IDX && wb + lane < we) ? tile_row(p, prefix, wb + lane) : 0;
   long long nx_base = wb + 32;
   int nx_row = (!IDX && nx_base + lane < we) ? tile_row(p, prefix, nx_base + lane) : 0;
-  int idx_row = (IDX && wb < we) ? indexed_row(p, prefix, wb, lane & 15) : -2;
+  IdxLookup idx;
+  if (IDX)                               // fill the chain: tile wb at its end
+    for (int x = 0; x < 3; ++x) idx_advance(p, prefix, idx, wb + x, we, lane & 15);
   long long issued = wb;                              // next tile to issue
 
   // Issue tile `issued` into its stage (lane 0 does the copy; all lanes call).
   auto issue_next = [&]() {
     if (issued >= we) return;
     if (IDX) {
-      // gather: lane l copies half of selected row l % 16 (K and V), 16 bytes per
-      // cp.async, into the swizzled layout the TMA path produces
+      // gather: instruction x copies selected rows 2x and 2x + 1 whole, one per
+      // half-warp, lane l taking 16-byte chunk l % 16 of its row (a row of K or V is
+      // 256 contiguous bytes, so each copy instruction reads 4 full 128-byte
+      // lines) into the swizzled layout the TMA path produces; lane r % 16 holds
+      // the row index of entry r and shares it
       const long long n = issued - wb;
       const int st = static_cast<int>(n % R);
+      const int idx_row = idx_row_of(p, idx);
       const bool bad = __any_sync(0xffffffffu, idx_row == -1);
-      if (!bad && idx_row >= 0) {
-        constexpr int kChunks = D / 8;                // 16-byte chunks per row
-        const int r = lane & 15, half = lane >> 4;
-        const char *ks = static_cast<const char *>(p.k_cache) + static_cast<long long>(idx_row) * D * 2;
-        const char *vs = static_cast<const char *>(p.v_cache) + static_cast<long long>(idx_row) * D * 2;
+      if (!bad) {
+        const int ch = lane & 15, hw = lane >> 4;
         const uint32_t dk = smem_u32(ring + st * L::kStage), dv = dk + L::kKTile;
 #pragma unroll
-        for (int cc = 0; cc < kChunks / 2; ++cc) {
-          const int ch = half * (kChunks / 2) + cc;
-          const uint32_t off = sw128_offset(r, ch * 8, kTile);
-          cp_async16(dk + off, ks + ch * 16);
-          cp_async16(dv + off, vs + ch * 16);
+        for (int x = 0; x < kTile / 2; ++x) {
+          const int r = 2 * x + hw;
+          const int row = __shfl_sync(0xffffffffu, idx_row, r);
+          if (row >= 0) {
+            const long long off = static_cast<long long>(row) * D * 2 + ch * 16;
+            const uint32_t so = sw128_offset(r, ch * 8, kTile);
+            cp_async16(dk + so, static_cast<const char *>(p.k_cache) + off);
+            cp_async16(dv + so, static_cast<const char *>(p.v_cache) + off);
+          }
         }
       }
       cp_async_mbar_arrive_noinc(&full[st]);
@@ -333,8 +369,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         mbar_arrive(&full[st]);
       }
       ++issued;
-      // the next tile's lookups now, so that their latency hides behind this tile
-      idx_row = issued < we ? indexed_row(p, prefix, issued, lane & 15) : -2;
+      idx_advance(p, prefix, idx, issued + 2, we, lane & 15);   // tile issued+2 enters
       return;
     }
     if (issued >= la_base + 32) {                     // slide the look-ahead window
