@@ -51,6 +51,8 @@ DESCRIPTIONS = {
     "mixed": "mixed continuous-batching decode: B256 Hq64 Hkv8 D128 bf16 bs16 ctx log-U[1,32768]",
     "gqa_fp8": "GQA decode over a float8 E4M3 KV cache (one scale per tensor): B32 Hq32 Hkv8 D128 "
                "bf16 q/out bs16 ctx U[512,4096] pool 1.25x shuffled",
+    "topk": "index-list GQA decode: B32 Hq32 Hkv8 D128 bf16 bs16 ctx 32768, 1152 selected "
+            "positions per sequence (1024 uniform + last 128), referenced blocks shuffled",
 }
 
 
@@ -59,7 +61,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="gqa", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="gqa",
+                    choices=sorted(list(workloads.WORKLOADS) + list(workloads.INDEXED)))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -105,13 +108,25 @@ def sum_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def get_workload(name, seed_offset=0):
+    import dataclasses
+    w = workloads.INDEXED[name] if name in workloads.INDEXED else workloads.get(name)
+    return dataclasses.replace(w, seed=w.seed + seed_offset) if seed_offset else w
+
+
+def make_inputs(w):
+    return workloads.make_indexed(w) if w.kind == "gqa_indexed" else workloads.make(w)
+
+
+def live_lens(w, inp):
+    """Tokens each sequence attends over (the selected counts for an index list)."""
+    return inp["n_sel"] if w.kind == "gqa_indexed" else inp["context_lens"]
+
+
 def rank_workload(name, rank, world):
     """The workload a rank decodes: the same shapes on every rank, its own seeded
     batch of independent sequences when several ranks run (weak scaling)."""
-    w = workloads.get(name)
-    if world > 1:
-        w = workloads.get(name, seed=w.seed + 7919 * rank)
-    return w
+    return get_workload(name, 7919 * rank if world > 1 else 0)
 
 
 def barrier(world):
@@ -216,6 +231,10 @@ def oracle_rows(w, inp, pairs, nthreads):
     import oracle
     u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
     bt, cl = inp["block_table"].numpy(), inp["context_lens"].numpy()
+    if w.kind == "gqa_indexed":
+        return oracle.decode_indexed(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]), bt,
+                                     inp["token_index"].numpy(), inp["n_sel"].numpy(),
+                                     inp["scale"], inp["dtype"], pairs=pairs, nthreads=nthreads)
     if w.kind == "gqa" and getattr(w, "kv_dtype", None) == "e4m3":
         return oracle.decode_kv8(u16(inp["q"]), inp["k_cache"].numpy(), inp["v_cache"].numpy(),
                                  inp["k_scale"], inp["v_scale"], bt, cl, inp["scale"],
@@ -231,8 +250,8 @@ def cpu_baseline(w, inp, target_s):
     """Time the float64 oracle on a bounded sample (leading sequences of the batch)."""
     import numpy as np
     nthreads = os.cpu_count() or 1
-    cl = inp["context_lens"]
-    H = w.num_q_heads if w.kind == "gqa" else w.num_heads
+    cl = live_lens(w, inp)
+    H = w.num_heads if w.kind == "mla" else w.num_q_heads
 
     def run(nseq, nheads):
         pairs = np.array([(b, h) for b in range(nseq) for h in range(nheads)], np.int32)
@@ -268,14 +287,25 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = rank_workload(args.workload, rank, world)
-    inp = workloads.make(w)
-    kv_bytes = workloads.kv_bytes(w, inp["context_lens"])
+    inp = make_inputs(w)
+    kv_bytes = workloads.kv_bytes(w, live_lens(w, inp))
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     scale = inp["scale"]
     stream = torch.cuda.current_stream(dev)
 
     kv8 = getattr(w, "kv_dtype", None) == "e4m3"
-    if w.kind == "gqa" and kv8:
+    if w.kind == "gqa_indexed":
+        desc = pa.gqa_desc(d["q"], d["k_cache"], d["block_table"])
+        out = torch.empty_like(d["q"])
+
+        def call(passes):
+            # the index-list entry point runs both passes
+            return pa.decode_indexed(d["q"], d["k_cache"], d["v_cache"], d["block_table"],
+                                     d["token_index"], d["n_sel"], scale, out=out, workspace=ws)
+        n_kernels = 1
+        kernel_files = ["pa_gqa.cuh", "pa_device.cuh"]
+        kname = "gqa_decode_kernel (index-list gathers)"
+    elif w.kind == "gqa" and kv8:
         desc = pa.PADesc(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
                          d["block_table"].shape[1], d["k_cache"].shape[0],
                          pa.PA_BF16 if w.dtype == "bf16" else pa.PA_F16, 0)
@@ -310,7 +340,8 @@ def run_ours(args, rank, world, local):
         kname = "mla_decode_kernel"
     ws = torch.empty(pa.workspace_size(desc), dtype=torch.uint8, device=dev)
     parts = desc.num_partitions or pa.default_partitions(
-        ("gqa_fp8" if kv8 else "gqa") if w.kind == "gqa" else "mla", getattr(w, "head_dim", 128))
+        {"gqa": "gqa_fp8" if kv8 else "gqa", "gqa_indexed": "gqa_indexed"}.get(w.kind, "mla"),
+        getattr(w, "head_dim", 128))
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -382,7 +413,11 @@ def run_ours(args, rank, world, local):
                 e0.record(stream)
             for k2, v in host.items():
                 dev_in[k2].copy_(v, non_blocking=True)
-            if w.kind == "gqa" and kv8:
+            if w.kind == "gqa_indexed":
+                pa.decode_indexed(dev_in["q"], dev_in["k_cache"], dev_in["v_cache"],
+                                  dev_in["block_table"], dev_in["token_index"], dev_in["n_sel"],
+                                  scale, out=out, workspace=ws)
+            elif w.kind == "gqa" and kv8:
                 pa.decode_kv8(dev_in["q"], dev_in["k_cache"], dev_in["v_cache"],
                               dev_in["block_table"], dev_in["context_lens"], scale,
                               inp["k_scale"], inp["v_scale"], out=out, workspace=ws)
@@ -429,7 +464,7 @@ def run_ours(args, rank, world, local):
         "dtype": inp["dtype"], "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool)",
         "config": {"workload": DESCRIPTIONS[args.workload], "batch": w.batch,
                    "kv_bytes_per_step_per_gpu": kv_bytes,
-                   "tokens_per_step_per_gpu": int(inp["context_lens"].sum()),
+                   "tokens_per_step_per_gpu": int(live_lens(w, inp).sum()),
                    "partitions": parts, "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed between steps (512 MiB write + 512 MiB read of another buffer)"},
         "roofline": roofline, "clocks": clocks, "e2e": e2e,
@@ -457,11 +492,11 @@ def run_reference(args, rank, world):
         return
     import numpy as np
 
-    w = workloads.get(args.workload)
-    inp = workloads.make(w)
+    w = get_workload(args.workload)
+    inp = make_inputs(w)
     nthreads = os.cpu_count() or 1
-    cl = inp["context_lens"]
-    H = w.num_q_heads if w.kind == "gqa" else w.num_heads
+    cl = live_lens(w, inp)
+    H = w.num_heads if w.kind == "mla" else w.num_q_heads
     # each step: a bounded sample (leading sequences, all heads) sized to ~2 s of CPU work
     budget_per_step = max(0.5, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
 
