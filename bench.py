@@ -71,6 +71,9 @@ def parse():
     ap.add_argument("--sweep", choices=["mha", "mqa"], default=None,
                     help="sequence-length scaling sweep 512..64k (one JSON line per length)")
     ap.add_argument("--sweep-batch", type=int, default=1)
+    ap.add_argument("--merge", choices=["separate", "fused"], default="separate",
+                    help="16-bit GQA workloads: 'fused' times pa_decode_fused (the last piece "
+                         "of each split segment merges it; one launch per step)")
     return ap.parse_args()
 
 
@@ -338,6 +341,12 @@ def run_ours(args, rank, world, local):
         n_kernels = 1
         kernel_files = ["pa_mla.cuh", "pa_tcgen05.cuh", "pa_device.cuh"]
         kname = "mla_decode_kernel"
+    fused = args.merge == "fused"
+    if fused and not (w.kind == "gqa" and not kv8):
+        raise SystemExit("--merge fused applies to the 16-bit GQA workloads")
+    step_passes = "fused" if fused else "both"
+    if fused:
+        kname = "gqa_decode_kernel (single-pass merge)"
     ws = torch.empty(pa.workspace_size(desc), dtype=torch.uint8, device=dev)
     parts = desc.num_partitions or pa.default_partitions(
         {"gqa": "gqa_fp8" if kv8 else "gqa", "gqa_indexed": "gqa_indexed"}.get(w.kind, "mla"),
@@ -352,7 +361,7 @@ def run_ours(args, rank, world, local):
 
     for _ in range(args.warmup):
         flush()
-        call("both")
+        call(step_passes)
     torch.cuda.synchronize()
     if pa.device_status() != 0:
         raise RuntimeError("kernel reported an error during warm-up")
@@ -370,7 +379,7 @@ def run_ours(args, rank, world, local):
     for i in range(K):
         flush()
         ev[i][0].record(stream)
-        call("both")
+        call(step_passes)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
@@ -378,14 +387,16 @@ def run_ours(args, rank, world, local):
     clocks = sampler.stop(t0, t1) if sampler else None
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     # the dominant kernel alone, for the roofline: same flush, events around the
-    # partition kernel only (the merge runs after the second event)
+    # partition kernel only (the merge runs after the second event; the
+    # single-pass form has no merge launch, its one kernel is timed)
     Kp = min(K, 200)
     for i in range(Kp):
         flush()
         ev[i][0].record(stream)
-        call("partition")
+        call("fused" if fused else "partition")
         ev[i][1].record(stream)
-        call("merge")
+        if not fused:
+            call("merge")
     torch.cuda.synchronize()
     part_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(Kp)]
     if pa.device_status() != 0:
@@ -423,7 +434,8 @@ def run_ours(args, rank, world, local):
                               inp["k_scale"], inp["v_scale"], out=out, workspace=ws)
             elif w.kind == "gqa":
                 pa.decode(dev_in["q"], dev_in["k_cache"], dev_in["v_cache"], dev_in["block_table"],
-                          dev_in["context_lens"], scale, out=out, workspace=ws)
+                          dev_in["context_lens"], scale, out=out, workspace=ws,
+                          passes=step_passes)
             else:
                 pa.decode_mla(dev_in["q"], dev_in["latent_cache"], dev_in["block_table"],
                               dev_in["context_lens"], scale, v_dim=w.v_dim, out=out, workspace=ws)
@@ -440,7 +452,8 @@ def run_ours(args, rank, world, local):
     part_avg_s = statistics.mean(part_ms) / 1e3
     achieved = kv_bytes / part_avg_s / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(args.workload, kernel_files),
+                "frac": round(achieved / hbm, 4),
+                "traffic": None if fused else profiled_traffic(args.workload, kernel_files),
                 "kernel": kname, "kernel_us": round(part_avg_s * 1e6, 2),
                 "peak_source": f"{peak_src} hbm_gbs (copy)",
                 "nominal_frac_8tbs": round(achieved / 8000.0, 4)}
@@ -465,11 +478,15 @@ def run_ours(args, rank, world, local):
         "config": {"workload": DESCRIPTIONS[args.workload], "batch": w.batch,
                    "kv_bytes_per_step_per_gpu": kv_bytes,
                    "tokens_per_step_per_gpu": int(live_lens(w, inp).sum()),
-                   "partitions": parts, "parallelism": f"replicas x{world} (independent batches)",
+                   "partitions": parts,
+                   "merge": ("single-pass (pa_decode_fused: one launch)" if fused else
+                             "separate kernel (programmatic dependent launch)"),
+                   "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed between steps (512 MiB write + 512 MiB read of another buffer)"},
         "roofline": roofline, "clocks": clocks, "e2e": e2e,
-        "gpu_launches": 2 * K,
-        "gpu_launches_note": "per step: the partition kernel + the LSE merge kernel",
+        "gpu_launches": (1 if fused else 2) * K,
+        "gpu_launches_note": ("per step: the partition kernel, which also merges" if fused else
+                              "per step: the partition kernel + the LSE merge kernel"),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(w, inp, args.cpu_seconds)

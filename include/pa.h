@@ -132,6 +132,26 @@ pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cach
                           const int32_t *context_lens, float scale, void *out, void *workspace,
                           size_t workspace_bytes, void *stream);
 
+/* pa_decode in one launch (single-pass merge): the same inputs, output and
+ * workspace as pa_decode, but no merge grid.  Each piece of a split
+ * (sequence, kv head) writes its normalised partial rows and log-sum-exps, then
+ * counts itself in at the segment's arrival counter in the workspace; the last
+ * piece to arrive merges the segment's rows with the same log-sum-exp
+ * arithmetic as pa_decode_merge (page "cidian.kuaisou.com: flash decoding ++":
+ * the per-block results are rescaled and combined once, at the end).
+ *
+ * The counters are tagged with a per-call epoch, so a workspace needs no
+ * clearing, and the last arrival resets its counter, so a call captured in a
+ * CUDA graph may be replayed.  The result equals pa_decode's up to the order of
+ * the merge's fp32 sums (the pieces are the same), and repeated calls on the
+ * same inputs are bitwise identical.  Two calls in flight at once must not share
+ * a workspace.  Errors as pa_decode; a call that reported PA_ERR_TIMEOUT may
+ * leave counters of its own epoch behind, which no later call reads. */
+pa_status pa_decode_fused(const pa_desc *desc, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *block_table,
+                          const int32_t *context_lens, float scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
 size_t pa_mla_workspace_size(const pa_mla_desc *desc);
 
 pa_status pa_decode_mla(const pa_mla_desc *desc, const void *q, const void *latent_cache,

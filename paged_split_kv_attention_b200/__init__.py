@@ -68,7 +68,7 @@ def library() -> ctypes.CDLL:
             vp, sz, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
             gqa = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp, f32, vp, vp, sz, vp]
             mla = [ctypes.POINTER(PAMLADesc), vp, vp, vp, vp, f32, vp, vp, sz, vp]
-            for name in ("pa_decode", "pa_decode_partition", "pa_decode_merge"):
+            for name in ("pa_decode", "pa_decode_partition", "pa_decode_merge", "pa_decode_fused"):
                 getattr(lib, name).argtypes = gqa
                 getattr(lib, name).restype = ctypes.c_int
             for name in ("pa_decode_mla", "pa_decode_mla_partition", "pa_decode_mla_merge"):
@@ -170,7 +170,8 @@ def _workspace(nbytes, device, workspace):
     return workspace
 
 
-_PASSES = {"both": "pa_decode", "partition": "pa_decode_partition", "merge": "pa_decode_merge"}
+_PASSES = {"both": "pa_decode", "partition": "pa_decode_partition", "merge": "pa_decode_merge",
+           "fused": "pa_decode_fused"}
 _MLA_PASSES = {"both": "pa_decode_mla", "partition": "pa_decode_mla_partition",
                "merge": "pa_decode_mla_merge"}
 
@@ -183,7 +184,9 @@ def decode(q, k_cache, v_cache, block_table, context_lens, scale, out=None, work
     block_table [B, max_blocks_per_seq] int32; context_lens [B] int32.
     Returns out [B, Hq, D] in q's dtype.  Asynchronous on the current stream.
     passes="partition" / "merge" run one of the two kernels (merge must follow
-    partition with the same arguments and workspace).
+    partition with the same arguments and workspace); passes="fused" is the
+    single-launch form (pa_decode_fused: the last piece of each split sequence
+    and kv head merges it).
     """
     _require(q, "q", ndim=3)
     _require(k_cache, "k_cache", q.dtype, 4)

@@ -97,8 +97,9 @@ int resident_ctas(const void *kernel, int threads, size_t smem) {
 
 // ------------------------------------------------------------------ GQA variants
 
-// Kernel modes: 16-bit cache, float8 cache, index-list decode.
-enum GqaMode { kMode16 = 0, kModeKv8 = 1, kModeIndexed = 2 };
+// Kernel modes: 16-bit cache, float8 cache, index-list decode, 16-bit cache with
+// the single-pass merge.
+enum GqaMode { kMode16 = 0, kModeKv8 = 1, kModeIndexed = 2, kModeFused = 3 };
 
 template <int D, int NT, bool BF16, int MODE>
 struct GqaVariant {
@@ -128,6 +129,9 @@ bool dispatch_gqa(int D, int NT, bool bf16, int mode, A &&...a) {
   PA_CASE(128, 2, false, 1)
   PA_CASE(128, 1, true, 2) PA_CASE(128, 1, false, 2) PA_CASE(128, 2, true, 2)
   PA_CASE(128, 2, false, 2)
+  PA_CASE(128, 1, true, 3) PA_CASE(128, 1, false, 3) PA_CASE(128, 2, true, 3)
+  PA_CASE(128, 2, false, 3) PA_CASE(64, 1, true, 3) PA_CASE(64, 1, false, 3)
+  PA_CASE(64, 2, true, 3) PA_CASE(64, 2, false, 3)
 #undef PA_CASE
   return false;
 }
@@ -142,7 +146,7 @@ struct QueryResident {
 
 struct GqaPlan {
   int G = 0, NT = 0, parts = 0;
-  size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
+  size_t off_prefix = 0, off_lse = 0, off_o = 0, off_ctr = 0, bytes = 0;
 };
 
 int default_gqa_parts(int D, int NT, bool bf16, int mode, int B) {
@@ -164,7 +168,7 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, int mode = kMode16) {
   const int G = d->num_q_heads / d->num_kv_heads;
   if (G > 16) return PA_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (mode != kMode16 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if ((mode == kModeKv8 || mode == kModeIndexed) && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (d->block_size % pa::kTile || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
   if (d->batch > kMaxBatch) return PA_ERR_UNSUPPORTED;
   const int64_t kv_rows = int64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
@@ -185,7 +189,9 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, int mode = kMode16) {
   pl->off_prefix = 0;
   pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
   pl->off_o = pl->off_lse + round_up(slots * G * 4, 256);
-  pl->bytes = pl->off_o + slots * G * size_t(d->head_dim) * 4;
+  // arrival counters of the single-pass merge, one 64-bit word per segment
+  pl->off_ctr = round_up(pl->off_o + slots * G * size_t(d->head_dim) * 4, 256);
+  pl->bytes = pl->off_ctr + size_t(d->batch) * d->num_kv_heads * 8;
   return PA_OK;
 }
 
@@ -290,7 +296,18 @@ constexpr int kMinTilesMla = 16;
 // their timeout path.
 std::atomic<int> g_stall_test{0};
 
-enum Pass { kPartition = 1, kMerge = 2, kBoth = 3 };
+// kFused: the partition kernel also merges (the last piece of each split segment),
+// so no merge grid is launched
+enum Pass { kPartition = 1, kMerge = 2, kBoth = 3, kFused = 4 };
+
+// Epoch of a single-pass call: tags the workspace's arrival counters so that words
+// left by another call (or never written) count as zero; never 0 (0 = not fused).
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> epoch{0};
+  uint32_t e;
+  do e = epoch.fetch_add(1, std::memory_order_relaxed) + 1; while (e == 0);
+  return e;
+}
 
 // mode kModeKv8: k / v hold float8 E4M3 codes, key = code x k_scale, value =
 // code x v_scale.  kModeIndexed: cl holds the selected counts and token_index
@@ -299,6 +316,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
                   const int32_t *bt, const int32_t *cl, float scale, void *out, void *ws,
                   size_t ws_bytes, void *stream, int mode = kMode16, float k_scale = 1.f,
                   float v_scale = 1.f, const int32_t *token_index = nullptr, int max_sel = 0) {
+  if (passes & kFused) mode = kModeFused;
   const bool kv8 = mode == kModeKv8;
   GqaPlan pl;
   pa_status s = plan_gqa(d, &pl, mode);
@@ -350,6 +368,8 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.v_cache = v;
     p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     p.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
+    p.seg_ctr = reinterpret_cast<unsigned long long *>(w + pl.off_ctr);
+    p.epoch = mode == kModeFused ? next_epoch() : 0u;
     cudaError_t err = cudaSuccess;
     if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, mode, pl.parts, st, maps, &p, &err))
       return PA_ERR_UNSUPPORTED;
@@ -502,9 +522,10 @@ size_t pa_workspace_size(const pa_desc *desc) {
   if (plan_gqa(desc, &pl) != PA_OK) return 0;
   size_t bytes = pl.bytes;
   // the float8 and index-list calls may launch another grid size
-  for (int mode : {kModeKv8, kModeIndexed}) {
+  for (int mode : {kModeKv8, kModeIndexed, kModeFused}) {
     GqaPlan other;
-    if (desc->head_dim == 128 && plan_gqa(desc, &other, mode) == PA_OK && other.bytes > bytes)
+    if ((mode == kModeFused || desc->head_dim == 128) && plan_gqa(desc, &other, mode) == PA_OK &&
+        other.bytes > bytes)
       bytes = other.bytes;
   }
   return bytes;
@@ -533,6 +554,14 @@ pa_status pa_decode(const pa_desc *desc, const void *q, const void *k_cache, con
                     void *out, void *workspace, size_t workspace_bytes, void *stream) {
   return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
                  workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_fused(const pa_desc *desc, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *block_table,
+                          const int32_t *context_lens, float scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+  return run_gqa(kPartition | kFused, desc, q, k_cache, v_cache, block_table, context_lens, scale,
+                 out, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_decode_partition(const pa_desc *desc, const void *q, const void *k_cache,

@@ -52,6 +52,7 @@
 #pragma once
 
 #include "pa_device.cuh"
+#include "pa_merge.cuh"
 
 namespace pa {
 
@@ -78,10 +79,13 @@ struct GqaParams {
   const int32_t *token_index;   // [B][max_sel] token positions
   int max_sel;
   const void *k_cache, *v_cache;  // the gathers read the caches directly
+  // single-pass merge: nonzero epoch = the last piece of a split segment merges it
+  unsigned long long *seg_ctr;  // [B * Hkv] arrival counters (epoch << 32 | count)
+  uint32_t epoch;
 };
 
-// MODE 0 and 2: 16-bit rows in 128-byte swizzled slabs (2: gathered row by row
-// into the same layout).  MODE 1: float8 rows.
+// MODE 0, 2 and 3: 16-bit rows in 128-byte swizzled slabs (2: gathered row by
+// row into the same layout).  MODE 1: float8 rows.
 template <int D, int NT, int R, int MODE = 0>
 struct GqaLayout {
   static constexpr int kHeads = 8 * NT;            // group width padded to the MMA N
@@ -249,11 +253,12 @@ __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int l
 
 // MODE 0: 16-bit cache, TMA tiles.  1: float8 cache (KV8).  2: index-list
 // decode (IDX): each warp gathers its tiles' selected rows with cp.async.
+// 3: as 0, and the last piece of each split segment merges it (FUSED).
 template <int D, int NT, bool BF16, int R, int MODE = 0>
 __global__ void __launch_bounds__(kGqaThreads, 1)
 gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
-  constexpr bool KV8 = MODE == 1, IDX = MODE == 2;
+  constexpr bool KV8 = MODE == 1, IDX = MODE == 2, FUSED = MODE == 3;
   using L = GqaLayout<D, NT, R, MODE>;
   static_assert(!KV8 || D == 128, "the float8 KV path reads 128-byte rows");
   static_assert(!IDX || D == 128, "index-list gathers read 256-byte rows");
@@ -624,6 +629,13 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (!whole && g == 0)
           p.part_lse[slot * p.G + h] = l[nt][e] > 0.f ? m[nt][e] + log2f(l[nt][e]) : -INFINITY;
       }
+    if (FUSED && !whole && !aborted) {
+      const int g0 = piece_of(seg_first, TP, pieces), g1 = piece_of(seg_first + P - 1, TP, pieces);
+      const int expected = pieces_with_tiles(g0, g1, TP, pieces, lane);
+      if (segment_arrive_last(p.seg_ctr + seg, p.epoch, expected, lane))
+        merge_segment_warp<D, 8 * NT, BF16>(p.part_o, p.part_lse, seg, p.G, g0, g1, TP, pieces,
+                                           orow, lane);
+    }
     // advance to the next segment
     b = nb_;
     kvh = nkvh;

@@ -189,3 +189,177 @@ merge_rows_kernel(const MergeParams p) {
 }
 
 }  // namespace pa
+
+namespace pa {
+
+// ---------------------------------------------------------------- fused merge
+//
+// Single-pass form (the partition kernel merges, no second launch): every piece
+// of a split segment, after writing its partial rows, arrives at the segment's
+// counter in the workspace; the last of the segment's pieces to arrive merges
+// all G rows of the segment with the arithmetic above and writes the output.
+//
+// A counter is a 64-bit word (call epoch << 32 | arrivals).  A word whose epoch
+// is not this call's counts as zero, so a workspace needs no clearing before its
+// first call; the last arrival also stores 0, so replays of a captured call
+// (same epoch) start from zero too.  The count is taken with compare-and-swap:
+// each failed attempt means another piece got in, so the loop ends after at most
+// as many rounds as the segment has pieces (bounded besides, as every wait here).
+
+// Lane 0 arrives; the warp learns whether it was the last of `expected`.
+__device__ __forceinline__ bool segment_arrive_last(unsigned long long *ctr, uint32_t epoch,
+                                                    int expected, int lane) {
+  int last = 0;
+  __threadfence();                        // every lane's partial rows before the arrival
+  __syncwarp();
+  if (lane == 0) {
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(ctr);
+    unsigned long long nw = 0;
+    bool done = false;
+    for (int it = 0; it < (1 << 20); ++it) {
+      const uint32_t cnt = static_cast<uint32_t>(old >> 32) == epoch ? static_cast<uint32_t>(old) : 0u;
+      nw = (static_cast<unsigned long long>(epoch) << 32) | (cnt + 1u);
+      const unsigned long long got = atomicCAS(ctr, old, nw);
+      if (got == old) {
+        done = true;
+        break;
+      }
+      old = got;
+    }
+    if (!done) record_error(5 /* PA_ERR_TIMEOUT */);
+    last = done && static_cast<int>(static_cast<uint32_t>(nw)) == expected;
+    if (last) *reinterpret_cast<volatile unsigned long long *>(ctr) = 0ull;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (last) __threadfence();              // the other pieces' rows after their arrivals
+  return last != 0;
+}
+
+// Non-empty pieces among g0..g1 (an explicit partition count can exceed the
+// tiles, and an empty piece writes nothing).
+__device__ __forceinline__ int pieces_with_tiles(int g0, int g1, long long TP, int pieces,
+                                                 int lane) {
+  int n = 0;
+  for (int pc = g0 + lane; pc <= g1; pc += 32)
+    n += piece_begin(pc + 1, TP, pieces) > piece_begin(pc, TP, pieces);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+  return n;
+}
+
+// One warp merges segment `seg` (pieces g0..g1, G <= GH rows of D) into out_rows
+// (the segment's G output rows, 16-bit), eight rows at a time.  Lane l holds the
+// weights of piece base + l for the eight rows; float4 i = l + 32k of the rows'
+// part of a piece's [G][D] partial block belongs to row i / (D/4) of the eight:
+// row k for D = 128, row 2k + l/16 for D = 64.
+template <int D, int GH, bool BF16>
+__device__ __forceinline__ void merge_segment_warp(const float *part_o, const float *part_lse,
+                                                   long long seg, int G, int g0, int g1,
+                                                   long long TP, int pieces, uint16_t *out_rows,
+                                                   int lane) {
+  static_assert(D == 64 || D == 128, "head dims 64 and 128");
+  static_assert(GH % 8 == 0, "rows in chunks of eight");
+  constexpr int F4 = D / 4;                         // float4 per row
+  constexpr int K4 = 8 * F4 / 32;                   // float4 per lane per piece and chunk
+  constexpr int kU = 2;                             // pieces whose loads are in flight together
+  const int n4 = G * F4;                            // float4 per piece block
+  auto lse_at = [&](int pc, int h) {
+    return __ldcg(&part_lse[(static_cast<long long>(pc) + seg) * G + h]);
+  };
+  auto nonempty = [&](int pc) {
+    return pc <= g1 && piece_begin(pc + 1, TP, pieces) > piece_begin(pc, TP, pieces);
+  };
+  // log-sum-exps of the first 32 pieces stay in registers for the weights
+  float L0[GH], M[GH];
+  const bool mine0 = nonempty(g0 + lane);
+#pragma unroll
+  for (int h = 0; h < GH; ++h) L0[h] = (mine0 && h < G) ? lse_at(g0 + lane, h) : -INFINITY;
+#pragma unroll
+  for (int h = 0; h < GH; ++h) M[h] = L0[h];
+  for (int pc = g0 + 32 + lane; pc <= g1; pc += 32)
+    if (nonempty(pc))
+#pragma unroll
+      for (int h = 0; h < GH; ++h)
+        if (h < G) M[h] = fmaxf(M[h], lse_at(pc, h));
+#pragma unroll
+  for (int h = 0; h < GH; ++h)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(0xffffffffu, M[h], off));
+
+#pragma unroll
+  for (int hc = 0; hc < GH / 8; ++hc) {
+    if (8 * hc >= G) break;
+    const int c0 = 8 * hc * F4;                     // first float4 of the chunk's rows
+    float4 acc[K4];
+#pragma unroll
+    for (int k = 0; k < K4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float W[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) W[j] = 0.f;
+    for (int base = g0; base <= g1; base += 32) {
+      float wl[8];
+      const bool mine = nonempty(base + lane);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int h = 8 * hc + j;
+        wl[j] = (mine && h < G)
+                    ? exp2f((base == g0 ? L0[h] : lse_at(base + lane, h)) - M[h]) : 0.f;
+      }
+      const int n = min(32, g1 - base + 1);
+      const unsigned ne = __ballot_sync(0xffffffffu, mine);
+      // kU pieces per round, their loads issued together; an empty piece (or one
+      // past the end) has weight 0 and loads nothing
+      for (int i = 0; i < n; i += kU) {
+        float4 v[kU][K4];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const bool e = i + u < n && ((ne >> (i + u)) & 1u);
+          const float4 *blk = reinterpret_cast<const float4 *>(
+              part_o + (static_cast<long long>(base + i + u) + seg) * G * D) + c0;
+#pragma unroll
+          for (int k = 0; k < K4; ++k)
+            v[u][k] = (e && c0 + lane + 32 * k < n4) ? __ldcg(blk + lane + 32 * k)
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int src = (i + u) & 31;
+          const bool in = i + u < n;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = __shfl_sync(0xffffffffu, wl[j], src);
+            W[j] += in ? x : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < K4; ++k) {
+            float w;
+            if (D == 128) {
+              w = __shfl_sync(0xffffffffu, wl[k], src);
+            } else {
+              const float wa = __shfl_sync(0xffffffffu, wl[2 * k], src);
+              const float wb = __shfl_sync(0xffffffffu, wl[2 * k + 1], src);
+              w = (lane >> 4) ? wb : wa;
+            }
+            w = in ? w : 0.f;
+            acc[k].x += w * v[u][k].x;
+            acc[k].y += w * v[u][k].y;
+            acc[k].z += w * v[u][k].z;
+            acc[k].w += w * v[u][k].w;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < K4; ++k) {
+      const int i4 = c0 + lane + 32 * k;
+      if (i4 >= n4) continue;
+      const float Wr = D == 128 ? W[k] : ((lane >> 4) ? W[2 * k + 1] : W[2 * k]);
+      const float inv = Wr > 0.f ? 1.f / Wr : 0.f;
+      *reinterpret_cast<uint2 *>(out_rows + 4 * i4) =
+          make_uint2(pack2<BF16>(acc[k].x * inv, acc[k].y * inv),
+                     pack2<BF16>(acc[k].z * inv, acc[k].w * inv));
+    }
+  }
+}
+
+}  // namespace pa

@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("pa_decode", "pa_decode_mla", "pa_workspace_size", "pa_mla_workspace_size",
                  "pa_decode_partition", "pa_decode_merge", "pa_decode_mla_partition",
-                 "pa_decode_mla_merge", "pa_device_status",
+                 "pa_decode_mla_merge", "pa_decode_fused", "pa_device_status",
                  "pa_status_string"):
         assert want in names, names
 
