@@ -429,6 +429,9 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   int ctx = clamp_ctx(__ldg(&p.context_lens[b]), cap);
   bool aborted = false;
 
+  long long split_seg[2] = {0, 0}, split_first[2] = {0, 0};
+  int split_tiles[2] = {0, 0}, n_split = 0;
+
   long long t = wb;
   while (t < we) {
     const int P = prefix[b + 1] - prefix[b];
@@ -629,12 +632,13 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (!whole && g == 0)
           p.part_lse[slot * p.G + h] = l[nt][e] > 0.f ? m[nt][e] + log2f(l[nt][e]) : -INFINITY;
       }
-    if (FUSED && !whole && !aborted) {
-      const int g0 = piece_of(seg_first, TP, pieces), g1 = piece_of(seg_first + P - 1, TP, pieces);
-      const int expected = pieces_with_tiles(g0, g1, TP, pieces, lane);
-      if (segment_arrive_last(p.seg_ctr + seg, p.epoch, expected, lane))
-        merge_segment_warp<D, 8 * NT, BF16>(p.part_o, p.part_lse, seg, p.G, g0, g1, TP, pieces,
-                                           orow, lane);
+    // single-pass merge: only a piece's first and last segments can be split;
+    // their arrivals wait until the piece is done, off the streaming path
+    if (FUSED && !whole && n_split < 2) {
+      split_seg[n_split] = seg;
+      split_first[n_split] = seg_first;
+      split_tiles[n_split] = P;
+      ++n_split;
     }
     // advance to the next segment
     b = nb_;
@@ -647,6 +651,25 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         qf[nt][ks][0] = nq[nt][ks][0];
         qf[nt][ks][1] = nq[nt][ks][1];
       }
+  }
+
+  if (FUSED && n_split > 0 && !aborted) {
+    __threadfence();                     // every lane's partial rows before the arrivals
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (i >= n_split) break;
+      const long long sg = split_seg[i];
+      const int g0 = piece_of(split_first[i], TP, pieces);
+      const int g1 = piece_of(split_first[i] + split_tiles[i] - 1, TP, pieces);
+      const int expected = pieces_with_tiles(g0, g1, TP, pieces, lane);
+      if (segment_arrive_last(p.seg_ctr + sg, p.epoch, expected, lane)) {
+        const long long sb = sg / p.Hkv, skv = sg - sb * p.Hkv;
+        uint16_t *rows = reinterpret_cast<uint16_t *>(p.out) + (sb * p.Hq + skv * p.G) * D;
+        merge_segment_warp<D, 8 * NT, BF16>(p.part_o, p.part_lse, sg, p.G, g0, g1, TP, pieces,
+                                           rows, lane);
+      }
+    }
   }
 
   if (aborted && lane == 0) {

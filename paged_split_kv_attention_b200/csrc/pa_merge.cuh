@@ -206,12 +206,11 @@ namespace pa {
 // each failed attempt means another piece got in, so the loop ends after at most
 // as many rounds as the segment has pieces (bounded besides, as every wait here).
 
-// Lane 0 arrives; the warp learns whether it was the last of `expected`.
+// Lane 0 arrives; the warp learns whether it was the last of `expected`.  The
+// caller has fenced its partial rows (every lane) before the first arrival.
 __device__ __forceinline__ bool segment_arrive_last(unsigned long long *ctr, uint32_t epoch,
                                                     int expected, int lane) {
   int last = 0;
-  __threadfence();                        // every lane's partial rows before the arrival
-  __syncwarp();
   if (lane == 0) {
     unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(ctr);
     unsigned long long nw = 0;
