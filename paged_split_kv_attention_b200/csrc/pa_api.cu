@@ -146,7 +146,7 @@ struct QueryResident {
 
 struct GqaPlan {
   int G = 0, NT = 0, parts = 0;
-  size_t off_prefix = 0, off_lse = 0, off_o = 0, off_ctr = 0, bytes = 0;
+  size_t off_lse = 0, off_o = 0, off_ctr = 0, bytes = 0;
 };
 
 int default_gqa_parts(int D, int NT, bool bf16, int mode, int B) {
@@ -186,8 +186,7 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, int mode = kMode16) {
   }
   // one partial slot per (warp piece, segment) pair a piece can end: piece + segment
   const size_t slots = size_t(pl->parts) * pa::kWarps + size_t(d->batch) * d->num_kv_heads;
-  pl->off_prefix = 0;
-  pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
+  pl->off_lse = 0;
   pl->off_o = pl->off_lse + round_up(slots * G * 4, 256);
   // arrival counters of the single-pass merge, one 64-bit word per segment
   pl->off_ctr = round_up(pl->off_o + slots * G * size_t(d->head_dim) * 4, 256);
@@ -230,7 +229,7 @@ cudaError_t launch_merge(const pa::MergeParams &mp, int segments, cudaStream_t s
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(segments), static_cast<unsigned>(mp.G), 1);
   cfg.blockDim = dim3(pa::kMergeThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = pa::merge_smem_bytes(mp.B);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -248,7 +247,7 @@ cudaError_t launch_merge_rows(const pa::MergeParams &mp, int segments, cudaStrea
   cfg.gridDim = dim3(static_cast<unsigned>((rows + pa::kMergeRowsPerCta - 1) / pa::kMergeRowsPerCta),
                      1, 1);
   cfg.blockDim = dim3(pa::kMergeRowsPerCta * 32, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = pa::merge_smem_bytes(mp.B);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -350,7 +349,6 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.out = out;
     p.part_o = reinterpret_cast<float *>(w + pl.off_o);
     p.part_lse = reinterpret_cast<float *>(w + pl.off_lse);
-    p.prefix_out = reinterpret_cast<int32_t *>(w + pl.off_prefix);
     p.B = d->batch;
     p.Hq = d->num_q_heads;
     p.Hkv = d->num_kv_heads;
@@ -379,7 +377,9 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     pa::MergeParams mp;
     mp.part_o = reinterpret_cast<const float *>(w + pl.off_o);
     mp.part_lse = reinterpret_cast<const float *>(w + pl.off_lse);
-    mp.prefix = reinterpret_cast<const int32_t *>(w + pl.off_prefix);
+    mp.lens = cl;
+    mp.cap = mode == kModeIndexed ? max_sel : d->max_blocks_per_seq * d->block_size;
+    mp.tile = pa::kTile;
     mp.out = out;
     mp.B = d->batch;
     mp.Hq = d->num_q_heads;
@@ -398,7 +398,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
 
 struct MlaPlan {
   int parts = 0;
-  size_t off_prefix = 0, off_lse = 0, off_o = 0, bytes = 0;
+  size_t off_lse = 0, off_o = 0, bytes = 0;
 };
 
 // Pieces whose two CTAs can all be resident at once (one CTA per SM).
@@ -438,8 +438,7 @@ pa_status plan_mla(const pa_mla_desc *d, MlaPlan *pl) {
     if (pl->parts <= 0) return PA_ERR_CUDA;
   }
   const size_t slots = size_t(pl->parts) + size_t(d->batch);
-  pl->off_prefix = 0;
-  pl->off_lse = round_up(size_t(d->batch + 1) * 4, 256);
+  pl->off_lse = 0;
   pl->off_o = pl->off_lse + round_up(slots * pa::kMlaHeads * 4, 256);
   pl->bytes = pl->off_o + slots * pa::kMlaHeads * size_t(pa::kMlaDv) * 4;
   return PA_OK;
@@ -473,7 +472,6 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     p.out = out;
     p.part_o = reinterpret_cast<float *>(w + pl.off_o);
     p.part_lse = reinterpret_cast<float *>(w + pl.off_lse);
-    p.prefix_out = reinterpret_cast<int32_t *>(w + pl.off_prefix);
     p.B = d->batch;
     p.bs = d->block_size;
     p.mbs = d->max_blocks_per_seq;
@@ -497,7 +495,9 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     pa::MergeParams mp;
     mp.part_o = reinterpret_cast<const float *>(w + pl.off_o);
     mp.part_lse = reinterpret_cast<const float *>(w + pl.off_lse);
-    mp.prefix = reinterpret_cast<const int32_t *>(w + pl.off_prefix);
+    mp.lens = cl;
+    mp.cap = d->max_blocks_per_seq * d->block_size;
+    mp.tile = pa::kMlaTile;
     mp.out = out;
     mp.B = d->batch;
     mp.Hq = pa::kMlaHeads;

@@ -221,6 +221,40 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows) {
                                ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
 
+__device__ __forceinline__ int clamp_ctx(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
+
+// prefix[0] = 0, prefix[b + 1] = sum_{b' <= b} ceil(clamp(ctx[b']) / tile).  All threads.
+template <int NTHREADS>
+__device__ void tiles_prefix(const int32_t *ctx, int B, int cap, int tile, int *prefix,
+                             int *scratch, bool report) {
+  const int per = (B + NTHREADS - 1) / NTHREADS;
+  const int b0 = threadIdx.x * per;
+  const int b1 = min(B, b0 + per);
+  int local = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int c = ctx[b];
+    if (report && (c < 0 || c > cap)) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
+    local += (clamp_ctx(c, cap) + tile - 1) / tile;
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) scratch[w] = v;
+  __syncthreads();
+  int run = v - local;
+  for (int i = 0; i < w; ++i) run += scratch[i];
+  if (threadIdx.x == 0) prefix[0] = 0;
+  for (int b = b0; b < b1; ++b) {
+    run += (clamp_ctx(ctx[b], cap) + tile - 1) / tile;
+    prefix[b + 1] = run;
+  }
+  __syncthreads();
+}
+
 // Partition of a flattened work stream of `total` units into `parts` equal
 // pieces: piece c covers [begin(c), begin(c + 1)).
 __device__ __forceinline__ long long piece_begin(long long c, long long total, long long parts) {

@@ -67,7 +67,6 @@ struct GqaParams {
   void *out;                    // [B][Hq][D] 16-bit
   float *part_o;                // [slots][G][D]
   float *part_lse;              // [slots][G], log2 units
-  int32_t *prefix_out;          // [B+1] tiles per kv head (written by CTA 0 for the merge)
   int B, Hq, Hkv, G, bs, mbs, nb;
   int tiles_per_block;          // bs / 16
   int parts;                    // gridDim.x
@@ -102,39 +101,6 @@ struct GqaLayout {
   static_assert(bars % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
-__device__ __forceinline__ int clamp_ctx(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
-
-// prefix[0] = 0, prefix[b + 1] = sum_{b' <= b} ceil(clamp(ctx[b']) / tile).  All threads.
-template <int NTHREADS>
-__device__ void tiles_prefix(const int32_t *ctx, int B, int cap, int tile, int *prefix,
-                             int *scratch, bool report) {
-  const int per = (B + NTHREADS - 1) / NTHREADS;
-  const int b0 = threadIdx.x * per;
-  const int b1 = min(B, b0 + per);
-  int local = 0;
-  for (int b = b0; b < b1; ++b) {
-    const int c = ctx[b];
-    if (report && (c < 0 || c > cap)) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
-    local += (clamp_ctx(c, cap) + tile - 1) / tile;
-  }
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int v = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
-  }
-  if (lane == 31) scratch[w] = v;
-  __syncthreads();
-  int run = v - local;
-  for (int i = 0; i < w; ++i) run += scratch[i];
-  if (threadIdx.x == 0) prefix[0] = 0;
-  for (int b = b0; b < b1; ++b) {
-    run += (clamp_ctx(ctx[b], cap) + tile - 1) / tile;
-    prefix[b + 1] = run;
-  }
-  __syncthreads();
-}
 
 // Segment (b, kvh) and tile j within it of flattened tile t (0 <= t < Hkv * prefix[B]).
 __device__ __forceinline__ void locate_tile(const int *prefix, int B, int Hkv, long long t,
@@ -285,8 +251,6 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + off));
   }
   tiles_prefix<kGqaThreads>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0);
-  if (c == 0)
-    for (int i = tid; i <= p.B; i += kGqaThreads) p.prefix_out[i] = prefix[i];
   // let the merge grid be scheduled as SMs free up (it waits for this grid to finish)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // sequences with no tokens get an all-zero output row (spread over the grid)

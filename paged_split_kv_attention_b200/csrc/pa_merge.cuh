@@ -17,7 +17,9 @@
 // sums meet in shared memory.  Segments covered by a single piece were written
 // by the partition pass and are skipped.  The kernel is launched with
 // programmatic dependent launch: its CTAs may be scheduled while the partition
-// grid drains and wait on griddepcontrol before reading its results.
+// grid drains.  Each CTA first derives the tile prefix (and so which pieces
+// cover its rows) from the sequence lengths, an input, then waits on
+// griddepcontrol before reading the partition pass's results.
 #pragma once
 
 #include "pa_device.cuh"
@@ -27,7 +29,8 @@ namespace pa {
 struct MergeParams {
   const float *part_o;       // [slots][G][DV]
   const float *part_lse;     // [slots][G]
-  const int32_t *prefix;     // [B + 1] tiles per kv head (written by the partition pass)
+  const int32_t *lens;       // [B] the partition pass's sequence lengths (tokens)
+  int cap, tile;             // its length clamp and tokens per tile
   void *out;                 // [B][Hq][DV] 16-bit
   int B, Hq, Hkv, G;
   int pieces;                // pieces launched by the partition pass
@@ -36,6 +39,11 @@ struct MergeParams {
 };
 
 constexpr int kMergeThreads = 256;
+
+// Dynamic shared memory of a merge CTA: the tile prefix [B + 1] and scan scratch.
+__host__ __device__ constexpr size_t merge_smem_bytes(int B) {
+  return static_cast<size_t>(B + 1 + 8) * 4;
+}
 
 template <int DV, bool BF16>
 __global__ void __launch_bounds__(kMergeThreads)
@@ -46,19 +54,23 @@ merge_kernel(const MergeParams p) {
   __shared__ float red[kMergeThreads / 32];
   __shared__ float4 acc_s[PG][TPR];
   __shared__ float w_s[PG];
+  extern __shared__ int merge_prefix[];      // [B + 1], then 8 ints of scan scratch
 
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
+  tiles_prefix<kMergeThreads>(p.lens, p.B, p.cap, p.tile, merge_prefix,
+                              merge_prefix + p.B + 1, false);
+  const int *prefix = merge_prefix;
   const int seg = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int b = seg / p.Hkv, kvh = seg - (seg / p.Hkv) * p.Hkv;
-  const int P = p.prefix[b + 1] - p.prefix[b];
+  const int P = prefix[b + 1] - prefix[b];
   if (P <= 0 || h >= p.G) return;
-  const long long TP = static_cast<long long>(p.Hkv) * p.prefix[p.B];
+  const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
   const int pieces = used_pieces(p.pieces, TP, p.min_tiles, p.floor_pieces);
-  const long long first = static_cast<long long>(p.Hkv) * p.prefix[b] + static_cast<long long>(kvh) * P;
+  const long long first = static_cast<long long>(p.Hkv) * prefix[b] + static_cast<long long>(kvh) * P;
   const int g0 = piece_of(first, TP, pieces);
   const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // M = max over the pieces that own tiles (an empty piece wrote nothing)
   float M = -INFINITY;
@@ -125,21 +137,26 @@ __global__ void __launch_bounds__(kMergeRowsPerCta * 32)
 merge_rows_kernel(const MergeParams p) {
   constexpr int V4 = DV / 128;                   // float4 columns per lane
   static_assert(V4 * 128 == DV, "DV must be a multiple of 128");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ int merge_prefix[];          // [B + 1], then 8 ints of scan scratch
+  tiles_prefix<kMergeRowsPerCta * 32>(p.lens, p.B, p.cap, p.tile, merge_prefix,
+                                      merge_prefix + p.B + 1, false);
+  const int *prefix = merge_prefix;
   const int lane = threadIdx.x & 31;
   const long long r = static_cast<long long>(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
   const long long segs = static_cast<long long>(p.B) * p.Hkv;
   if (r >= segs * p.G) return;
   const int seg = static_cast<int>(r / p.G), h = static_cast<int>(r - static_cast<long long>(seg) * p.G);
   const int b = seg / p.Hkv, kvh = seg - (seg / p.Hkv) * p.Hkv;
-  const int P = p.prefix[b + 1] - p.prefix[b];
+  const int P = prefix[b + 1] - prefix[b];
   if (P <= 0) return;
-  const long long TP = static_cast<long long>(p.Hkv) * p.prefix[p.B];
+  const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
   const int pieces = used_pieces(p.pieces, TP, p.min_tiles, p.floor_pieces);
-  const long long first = static_cast<long long>(p.Hkv) * p.prefix[b] + static_cast<long long>(kvh) * P;
+  const long long first = static_cast<long long>(p.Hkv) * prefix[b] + static_cast<long long>(kvh) * P;
   const int g0 = piece_of(first, TP, pieces);
   const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // lse of the pieces that own tiles (an empty piece wrote nothing): -inf else
   auto lse_of = [&](int pc) {

@@ -71,7 +71,6 @@ struct MlaParams {
   void *out;                    // [B][128][512] bf16
   float *part_o;                // [slots][128][512]
   float *part_lse;              // [slots][128], log2 units
-  int32_t *prefix_out;          // [B+1] tiles per sequence, inclusive prefix (CTA 0 writes)
   int B, bs, mbs, nb;
   int parts;                    // pieces (two CTAs each)
   int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
@@ -213,7 +212,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
     const int pieces = used_pieces(p.parts, TP, p.min_tiles, p.B);
     tb = pair < pieces ? piece_begin(pair, TP, pieces) : 0;
     te = pair < pieces ? piece_begin(pair + 1, TP, pieces) : 0;
-    if (blockIdx.x == 0 && tid == 0) p.prefix_out[0] = 0;
     for (int b = b0; b < b1; ++b) {
       const int P = mla_tiles(__ldg(&p.context_lens[b]), cap);
       if (P > 0 && run <= tb && tb < run + P) {
@@ -221,7 +219,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
         start[1] = static_cast<int>(tb - run);
       }
       run += P;
-      if (blockIdx.x == 0) p.prefix_out[b + 1] = run;
     }
   }
   if (tid == 0) {
