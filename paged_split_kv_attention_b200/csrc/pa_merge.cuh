@@ -155,8 +155,60 @@ merge_rows_kernel(const MergeParams p) {
   const int g0 = piece_of(first, TP, pieces);
   const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
+  // which of the first 32 pieces own tiles (an empty piece wrote nothing)
+  const bool own_l = g0 + lane <= g1 &&
+                     piece_begin(g0 + lane + 1, TP, pieces) > piece_begin(g0 + lane, TP, pieces);
+  const unsigned own = __ballot_sync(0xffffffffu, own_l);
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // Few pieces: the log-sum-exps and every partial row are loaded in one round
+  // trip.  Empty pieces enter with weight 0 and a zero row, which leaves the
+  // sums exactly as the general loop below forms them.
+  constexpr int kFew = DV <= 128 ? 8 : 4;
+  if (g1 - g0 < kFew) {
+    const float l = own_l ? __ldcg(&p.part_lse[(static_cast<long long>(g0) + lane + seg) * p.G + h])
+                          : -INFINITY;
+    float4 v[kFew][V4];
+#pragma unroll
+    for (int i = 0; i < kFew; ++i) {
+      const bool e = (own >> i) & 1u;
+      const float4 *row = reinterpret_cast<const float4 *>(
+          p.part_o + ((static_cast<long long>(g0) + i + seg) * p.G + h) * DV);
+#pragma unroll
+      for (int k = 0; k < V4; ++k)
+        v[i][k] = e ? __ldcg(row + lane + 32 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float M = l;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float wl = own_l ? exp2f(l - M) : 0.f;
+    float4 acc[V4];
+#pragma unroll
+    for (int k = 0; k < V4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float W = 0.f;
+#pragma unroll
+    for (int i = 0; i < kFew; ++i) {
+      const float w = __shfl_sync(0xffffffffu, wl, i);
+      W += w;
+#pragma unroll
+      for (int k = 0; k < V4; ++k) {
+        acc[k].x += w * v[i][k].x;
+        acc[k].y += w * v[i][k].y;
+        acc[k].z += w * v[i][k].z;
+        acc[k].w += w * v[i][k].w;
+      }
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    uint16_t *o = reinterpret_cast<uint16_t *>(p.out) +
+                  (static_cast<long long>(b) * p.Hq + kvh * p.G + h) * DV;
+#pragma unroll
+    for (int k = 0; k < V4; ++k)
+      *reinterpret_cast<uint2 *>(o + 4 * (lane + 32 * k)) =
+          make_uint2(pack2<BF16>(acc[k].x * inv, acc[k].y * inv),
+                     pack2<BF16>(acc[k].z * inv, acc[k].w * inv));
+    return;
+  }
 
   // lse of the pieces that own tiles (an empty piece wrote nothing): -inf else
   auto lse_of = [&](int pc) {
