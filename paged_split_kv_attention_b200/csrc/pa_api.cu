@@ -62,6 +62,23 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t inner, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major [rows][128] 16-bit tensor viewed as (64 elements, rows, 2 halves),
+// the halves 128 bytes apart: one box of 64 x box_rows x 2 lands as
+// [2][box_rows][64] with 128 B swizzle, the layout two 64-wide 2-D boxes give.
+bool make_map_3d_halves(CUtensorMap *m, const void *base, bool bf16, uint64_t rows,
+                        uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {256, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Float8 KV cache: one byte per element, rows of `inner` bytes.
 bool make_map_2d_u8(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows,
                     uint32_t box_inner, uint32_t box_rows) {
@@ -339,6 +356,8 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     const bool mapped =
         kv8 ? make_map_2d_u8(&maps[0], k, D, kv_rows, D, pa::kTile) &&
                   make_map_2d_u8(&maps[1], v, D, kv_rows, D, pa::kTile)
+        : D == 128 ? make_map_3d_halves(&maps[0], k, bf16, kv_rows, pa::kTile) &&
+                         make_map_3d_halves(&maps[1], v, bf16, kv_rows, pa::kTile)
             : make_map_2d(&maps[0], k, bf16, D, kv_rows, 64, pa::kTile) &&
                   make_map_2d(&maps[1], v, bf16, D, kv_rows, 64, pa::kTile);
     if (!mapped) return PA_ERR_CUDA;

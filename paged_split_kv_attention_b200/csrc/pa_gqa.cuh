@@ -362,6 +362,11 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (KV8) {                                    // one 16 x 128-byte box each
           tma_load_2d_hint(dst, &tm_k, &full[st], 0, row, policy);
           tma_load_2d_hint(dst + L::kKTile, &tm_v, &full[st], 0, row, policy);
+        } else if (D == 128) {
+          // one box per tile: the row's two 128-byte halves are the map's third
+          // dimension, so the box lands as the two 64-wide swizzled slabs
+          tma_load_3d_hint(dst, &tm_k, &full[st], 0, row, 0, policy);
+          tma_load_3d_hint(dst + L::kKTile, &tm_v, &full[st], 0, row, 0, policy);
         } else {
 #pragma unroll
           for (int x = 0; x < D; x += 64) {
