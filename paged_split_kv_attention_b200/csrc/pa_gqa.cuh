@@ -443,10 +443,13 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
           const int c = 2 * x + (lane >> 4);
           return tile + x8_row * 128 + ((c ^ (x8_row & 7)) << 4);
         };
-        // S^T (16 tokens x 8NT heads) = K Q^T
-        float s[NT][4];
+        // S^T (16 tokens x 8NT heads) = K Q^T, the k-steps alternating between two
+        // accumulators (halves the chain of dependent MMAs), summed at the end
+        float s[NT][4], s2[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
         if (KV8) {
           // an ldmatrix block of 8 tokens x 16 codes gives lane (g, tq) the codes of
           // dims 4 tq .. 4 tq + 3 of token g: fragment columns (2tq, 2tq+1) and
@@ -462,7 +465,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
               e4m3x4_to_f16x2(r[2 * h + 1], a[1], a[3]);  // token g + 8
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
-                mma_16816<CT>(s[nt], a, qf[nt][2 * x + h][0], qf[nt][2 * x + h][1]);
+                mma_16816<CT>(h ? s2[nt] : s[nt], a, qf[nt][2 * x + h][0], qf[nt][2 * x + h][1]);
             }
           }
         } else {
@@ -471,9 +474,14 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             uint32_t a[4];
             ldsm_x4(kb + sw128_offset(k_row, ks * 16 + k_col, kTile), a);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_16816<CT>(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+            for (int nt = 0; nt < NT; ++nt)
+              mma_16816<CT>((ks & 1) ? s2[nt] : s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
           }
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
         // online softmax over the tile's tokens (rows g and g + 8 of this lane)
         const bool v0 = g < ntok, v1 = g + 8 < ntok;
         uint32_t pb[NT][2], pl[NT][2];
