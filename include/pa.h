@@ -76,9 +76,11 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 
 /* Shape of a GQA / MHA / MQA decode call.
  * Supported: head_dim in {64, 128}; block_size a multiple of 16 up to 1024;
- * 1 <= num_q_heads / num_kv_heads <= 16; batch >= 0 (0 is a no-op).
- * num_partitions: number of equal-work pieces the flattened KV stream is cut into
- * (one CTA each); 0 picks (SM count) x (resident CTAs per SM) for the current device. */
+ * 1 <= num_q_heads / num_kv_heads <= 16; 0 <= batch <= 4096 (0 is a no-op).
+ * num_partitions: CTAs of the partition grid; the flattened KV stream is cut into
+ * 8 equal-work pieces per CTA, one per warp.  0 picks (SM count) x (resident CTAs
+ * per SM) for the current device, with pieces no shorter than the partial output
+ * they write. */
 typedef struct {
   int batch;
   int num_q_heads;
@@ -92,7 +94,8 @@ typedef struct {
 } pa_desc;
 
 /* Shape of an MLA absorbed decode call.  Supported: num_heads 128, kv_dim 576,
- * v_dim 512, block_size a multiple of 32 up to 1024, dtype PA_BF16.
+ * v_dim 512, block_size a multiple of 32 up to 1024, dtype PA_BF16,
+ * 0 <= batch <= 32768.
  * num_partitions counts CTA pairs (0 = as many as can be resident). */
 typedef struct {
   int batch;

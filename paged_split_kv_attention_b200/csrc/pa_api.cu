@@ -21,6 +21,7 @@
 namespace {
 
 constexpr int kMaxBatch = 4096;            // prefix table lives in shared memory
+constexpr int kMaxBatchMla = 32768;        // the merge's prefix table: 128 KB of shared memory
 constexpr int kMaxPartitions = 1 << 20;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -241,8 +242,19 @@ struct LaunchPartition {
 
 // The merge kernel for value width DV, launched with programmatic dependent
 // launch so that its CTAs can be scheduled while the partition grid drains.
+// A merge CTA holds the tile prefix [B + 1] in dynamic shared memory; past the
+// 48 KB default the kernel's limit is raised first.
+cudaError_t merge_smem_limit(const void *kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes));
+}
+
 template <int DV, bool BF16>
 cudaError_t launch_merge(const pa::MergeParams &mp, int segments, cudaStream_t st) {
+  const cudaError_t e = merge_smem_limit(reinterpret_cast<const void *>(&pa::merge_kernel<DV, BF16>),
+                                         pa::merge_smem_bytes(mp.B));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(segments), static_cast<unsigned>(mp.G), 1);
   cfg.blockDim = dim3(pa::kMergeThreads, 1, 1);
@@ -259,6 +271,9 @@ cudaError_t launch_merge(const pa::MergeParams &mp, int segments, cudaStream_t s
 // Warp-per-row merge: one warp per (segment, head) row, 8 rows per CTA.
 template <int DV, bool BF16>
 cudaError_t launch_merge_rows(const pa::MergeParams &mp, int segments, cudaStream_t st) {
+  const cudaError_t e = merge_smem_limit(
+      reinterpret_cast<const void *>(&pa::merge_rows_kernel<DV, BF16>), pa::merge_smem_bytes(mp.B));
+  if (e != cudaSuccess) return e;
   const long long rows = static_cast<long long>(segments) * mp.G;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((rows + pa::kMergeRowsPerCta - 1) / pa::kMergeRowsPerCta),
@@ -447,6 +462,7 @@ pa_status plan_mla(const pa_mla_desc *d, MlaPlan *pl) {
       d->dtype != PA_BF16)
     return PA_ERR_UNSUPPORTED;
   if (d->block_size % pa::kMlaBox || d->block_size > 1024) return PA_ERR_UNSUPPORTED;
+  if (d->batch > kMaxBatchMla) return PA_ERR_UNSUPPORTED;
   const int64_t rows = int64_t(d->num_blocks) * d->block_size;
   const int64_t cap = int64_t(d->max_blocks_per_seq) * d->block_size;
   if (rows > INT32_MAX || cap > INT32_MAX || int64_t(d->batch) * pa::kMlaHeads > INT32_MAX)

@@ -98,3 +98,27 @@ def test_empty_batch_is_a_no_op(lib):
     d = _desc(batch=0)
     null = ctypes.c_void_p(0)
     assert lib.pa_decode(ctypes.byref(d), null, null, null, null, null, 0.1, null, null, 0, None) == 0
+
+
+def test_batch_limits(lib):
+    import paged_split_kv_attention_b200 as pa
+    z = ctypes.c_void_p(0x1000)
+    assert lib.pa_workspace_size(ctypes.byref(_desc(batch=4096))) > 0
+    big = _desc(batch=4097)
+    assert lib.pa_workspace_size(ctypes.byref(big)) == 0
+    assert lib.pa_decode(ctypes.byref(big), z, z, z, z, z, 0.1, z, z, 1 << 30, None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_fused(ctypes.byref(big), z, z, z, z, z, 0.1, z, z, 1 << 30,
+                               None) == pa.PA_ERR_UNSUPPORTED
+
+    def mla(batch):
+        return pa.PAMLADesc(batch, 128, 576, 512, 64, 32, 4096, pa.PA_BF16, 10)
+    assert lib.pa_mla_workspace_size(ctypes.byref(mla(32768))) > 0
+    assert lib.pa_mla_workspace_size(ctypes.byref(mla(32769))) == 0
+
+
+def test_fused_entry_point_rejects_what_pa_decode_rejects(lib):
+    z = ctypes.c_void_p(0x1000)
+    for bad in (dict(num_q_heads=30), dict(head_dim=96), dict(batch=-1)):
+        d = _desc(**bad)
+        assert (lib.pa_decode_fused(ctypes.byref(d), z, z, z, z, z, 0.1, z, z, 1 << 30, None) ==
+                lib.pa_decode(ctypes.byref(d), z, z, z, z, z, 0.1, z, z, 1 << 30, None) != 0)

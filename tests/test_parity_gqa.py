@@ -243,3 +243,23 @@ def test_full_size_long_sampled(dev):
 @pytest.mark.slow
 def test_full_size_mixed_sampled(dev):
     _sampled_full_size("mixed", dev)
+
+
+def test_maximum_batch(dev):
+    # 4096 sequences (the largest batch): the tile prefix of every kernel fills
+    # its shared-memory table; lengths 0..40 leave many segments unsplit and
+    # some empty
+    g = torch.Generator().manual_seed(11)
+    ctx = torch.randint(0, 41, (4096,), generator=g).tolist()
+    w = gqa(4096, 8, 2, 64, 16, ctx, seed=11)
+    inp = workloads.make(w)
+    d = to_dev(inp, dev)
+    out = run_gpu(d, inp["scale"])
+    rows = torch.randint(0, 4096, (40,), generator=g).tolist() + [4095, 0]
+    heads = torch.randint(0, 8, (42,), generator=g).tolist()
+    pairs = np.array(list(zip(rows, heads)), np.int32)
+    assert_close(out[pairs[:, 0], pairs[:, 1]], oracle_ref(inp, pairs=pairs), "B=4096")
+    for b in range(4096):
+        if ctx[b] == 0:
+            assert torch.all(out[b] == 0)
+            break

@@ -140,3 +140,31 @@ def test_full_size_mla_sampled(dev):
     pairs = np.array(list(zip(bs_, hs)), np.int32)
     ref = ref_of(inp, pairs=pairs)
     assert_close(out[pairs[:, 0], pairs[:, 1]], ref, "mla full")
+
+
+def test_batch_past_the_default_shared_memory_of_the_merge(dev):
+    # 13000 one-tile sequences: the merge's tile-prefix table (B + 1 ints) is past
+    # the 48 KB default, so the library raises the merge kernel's limit.  Inputs
+    # are drawn on the device (seeded); the oracle gets the sampled sequences only.
+    B, bs, H, Dk, Dv = 13000, 64, 128, 576, 512
+    gd = torch.Generator(device=dev).manual_seed(21)
+    q = torch.randn((B, H, Dk), generator=gd, device=dev).to(torch.bfloat16)
+    lat = torch.randn((B, bs, Dk), generator=gd, device=dev).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(21)
+    table = torch.randperm(B, generator=g).to(torch.int32).reshape(B, 1)
+    cl = torch.randint(1, bs + 1, (B,), generator=g).to(torch.int32)
+    scale = 1.0 / 192 ** 0.5
+    out = pa().decode_mla(q, lat, table.to(dev), cl.to(dev), scale, v_dim=Dv)
+    torch.cuda.synchronize()
+    assert pa().device_status() == 0
+    seqs = [0, B - 1] + torch.randint(0, B, (10,), generator=g).tolist()
+    blocks = table[seqs, 0].long()
+    q_s = q[seqs].cpu()
+    lat_s = lat[blocks.to(dev)].cpu()
+    table_s = torch.arange(len(seqs), dtype=torch.int32).reshape(-1, 1)
+    heads = torch.randint(0, H, (len(seqs),), generator=g).tolist()
+    pairs = np.array(list(zip(range(len(seqs)), heads)), np.int32)
+    ref = oracle.decode_mla(u16(q_s), u16(lat_s), table_s.numpy(), cl[seqs].numpy(), scale,
+                            "bf16", v_dim=Dv, pairs=pairs)
+    got = out[torch.tensor(seqs), torch.tensor(heads)]
+    assert_close(got, ref, "B=13000")
