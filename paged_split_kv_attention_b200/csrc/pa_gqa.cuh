@@ -404,6 +404,74 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   long long split_seg[2] = {0, 0}, split_first[2] = {0, 0};
   int split_tiles[2] = {0, 0}, n_split = 0;
 
+  // float8: per-lane row address of the ldmatrix blocks of a 16 x 128-byte
+  // tile (block j = lane / 8: tokens 8 (j & 1) .. +7, 16-byte chunk 2 x + j / 2)
+  const int x8_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+  auto x8_addr = [&](uint32_t tile, int x) {
+    const int c = 2 * x + (lane >> 4);
+    return tile + x8_row * 128 + ((c ^ (x8_row & 7)) << 4);
+  };
+  // scores S^T of the landed tile whose K starts at shared address kt
+  auto scores = [&](uint32_t kt, float (&sc)[NT][4]) {
+    // S^T (16 tokens x 8NT heads) = K Q^T, the k-steps alternating between two
+    // accumulators (halves the chain of dependent MMAs), summed at the end
+    float s2[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = s2[nt][e] = 0.f;
+    if (KV8) {
+      // an ldmatrix block of 8 tokens x 16 codes gives lane (g, tq) the codes of
+      // dims 4 tq .. 4 tq + 3 of token g: fragment columns (2tq, 2tq+1) and
+      // (2tq+8, 2tq+9) after widening (the query matches, see load_q)
+#pragma unroll
+      for (int x = 0; x < KS / 2; ++x) {
+        uint32_t r[4];
+        ldsm_x4(x8_addr(kt, x), r);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a[4];
+          e4m3x4_to_f16x2(r[2 * h], a[0], a[2]);      // token g
+          e4m3x4_to_f16x2(r[2 * h + 1], a[1], a[3]);  // token g + 8
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_16816<CT>(h ? s2[nt] : sc[nt], a, qf[nt][2 * x + h][0], qf[nt][2 * x + h][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(kt + sw128_offset(k_row, ks * 16 + k_col, kTile), a);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816<CT>((ks & 1) ? s2[nt] : sc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] += s2[nt][e];
+  };
+  // wait for the tile at position nn of the warp's run and take its scores
+  // (zeros for a tile that did not land or was not loaded)
+  auto land = [&](long long nn, float (&sc)[NT][4]) {
+    const int sst = static_cast<int>(nn % R);
+    const bool ok = !aborted && __all_sync(0xffffffffu, mbar_wait(&full[sst],
+                                                                  static_cast<uint32_t>((nn / R) & 1),
+                                                                  abort_flag));
+    if (!ok) aborted = true;
+    if (ok && stage_valid[sst]) {
+      scores(ring_base + sst * L::kStage, sc);
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+    }
+    return ok;
+  };
+
   long long t = wb;
   while (t < we) {
     const int P = prefix[b + 1] - prefix[b];
@@ -428,73 +496,6 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       for (int mt = 0; mt < KS; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
     }
 
-    // float8: per-lane row address of the ldmatrix blocks of a 16 x 128-byte
-    // tile (block j = lane / 8: tokens 8 (j & 1) .. +7, 16-byte chunk 2 x + j / 2)
-    const int x8_row = (lane & 7) + ((lane >> 3) & 1) * 8;
-    auto x8_addr = [&](uint32_t tile, int x) {
-      const int c = 2 * x + (lane >> 4);
-      return tile + x8_row * 128 + ((c ^ (x8_row & 7)) << 4);
-    };
-    // scores S^T of the landed tile whose K starts at shared address kt
-    auto scores = [&](uint32_t kt, float (&sc)[NT][4]) {
-      // S^T (16 tokens x 8NT heads) = K Q^T, the k-steps alternating between two
-      // accumulators (halves the chain of dependent MMAs), summed at the end
-      float s2[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] = s2[nt][e] = 0.f;
-      if (KV8) {
-        // an ldmatrix block of 8 tokens x 16 codes gives lane (g, tq) the codes of
-        // dims 4 tq .. 4 tq + 3 of token g: fragment columns (2tq, 2tq+1) and
-        // (2tq+8, 2tq+9) after widening (the query matches, see load_q)
-#pragma unroll
-        for (int x = 0; x < KS / 2; ++x) {
-          uint32_t r[4];
-          ldsm_x4(x8_addr(kt, x), r);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t a[4];
-            e4m3x4_to_f16x2(r[2 * h], a[0], a[2]);      // token g
-            e4m3x4_to_f16x2(r[2 * h + 1], a[1], a[3]);  // token g + 8
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              mma_16816<CT>(h ? s2[nt] : sc[nt], a, qf[nt][2 * x + h][0], qf[nt][2 * x + h][1]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t a[4];
-          ldsm_x4(kt + sw128_offset(k_row, ks * 16 + k_col, kTile), a);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_16816<CT>((ks & 1) ? s2[nt] : sc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] += s2[nt][e];
-    };
-    // wait for the tile at position nn of the warp's run and take its scores
-    // (zeros for a tile that did not land or was not loaded)
-    auto land = [&](long long nn, float (&sc)[NT][4]) {
-      const int sst = static_cast<int>(nn % R);
-      const bool ok = !aborted && __all_sync(0xffffffffu, mbar_wait(&full[sst],
-                                                                    static_cast<uint32_t>((nn / R) & 1),
-                                                                    abort_flag));
-      if (!ok) aborted = true;
-      if (ok && stage_valid[sst]) {
-        scores(ring_base + sst * L::kStage, sc);
-      } else {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-      }
-      return ok;
-    };
     // PIPE: tile t + 1's scores are taken before tile t's softmax and value MMA,
     // so each iteration holds two independent chains of MMAs.  Otherwise a tile
     // is waited for and scored in its own iteration.
