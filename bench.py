@@ -302,9 +302,9 @@ def run_ours(args, rank, world, local):
         out = torch.empty_like(d["q"])
 
         def call(passes):
-            # the index-list entry point runs both passes
             return pa.decode_indexed(d["q"], d["k_cache"], d["v_cache"], d["block_table"],
-                                     d["token_index"], d["n_sel"], scale, out=out, workspace=ws)
+                                     d["token_index"], d["n_sel"], scale, out=out, workspace=ws,
+                                     passes=passes)
         n_kernels = 1
         kernel_files = ["pa_gqa.cuh", "pa_device.cuh"]
         kname = "gqa_decode_kernel (index-list gathers)"
@@ -315,11 +315,9 @@ def run_ours(args, rank, world, local):
         out = torch.empty_like(d["q"])
 
         def call(passes):
-            # the float8 entry point runs both passes; a partition-only timing
-            # is not exposed for it
             return pa.decode_kv8(d["q"], d["k_cache"], d["v_cache"], d["block_table"],
                                  d["context_lens"], scale, inp["k_scale"], inp["v_scale"],
-                                 out=out, workspace=ws)
+                                 out=out, workspace=ws, passes=passes)
         n_kernels = 1
         kernel_files = ["pa_gqa.cuh", "pa_device.cuh"]
         kname = "gqa_decode_kernel (float8 KV)"

@@ -186,6 +186,19 @@ pa_status pa_decode_kv_e4m3(const pa_desc *desc, const void *q, const void *k_ca
                             const int32_t *context_lens, float scale, float k_scale,
                             float v_scale, void *out, void *workspace, size_t workspace_bytes,
                             void *stream);
+/* Its two passes on their own, as pa_decode_partition / pa_decode_merge: the
+ * merge must follow the partition pass on the same stream with the same
+ * arguments and workspace. */
+pa_status pa_decode_kv_e4m3_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_table,
+                                      const int32_t *context_lens, float scale, float k_scale,
+                                      float v_scale, void *out, void *workspace,
+                                      size_t workspace_bytes, void *stream);
+pa_status pa_decode_kv_e4m3_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_table,
+                                  const int32_t *context_lens, float scale, float k_scale,
+                                  float v_scale, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream);
 
 /* Index-list decode: each sequence attends over a given list of its token
  * positions instead of [0, context length), the dense kernel behind sparse
@@ -207,6 +220,18 @@ pa_status pa_decode_indexed(const pa_desc *desc, const void *q, const void *k_ca
                             const int32_t *token_index, int max_sel, const int32_t *n_sel,
                             float scale, void *out, void *workspace, size_t workspace_bytes,
                             void *stream);
+/* Its two passes on their own (the merge follows the partition pass on the same
+ * stream with the same arguments and workspace). */
+pa_status pa_decode_indexed_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_table,
+                                      const int32_t *token_index, int max_sel,
+                                      const int32_t *n_sel, float scale, void *out,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+pa_status pa_decode_indexed_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_table,
+                                  const int32_t *token_index, int max_sel, const int32_t *n_sel,
+                                  float scale, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream);
 
 /* Number of partitions (CTAs of the partition pass; each runs 8 independently
  * streaming warps, one piece each) a call with num_partitions == 0 uses on the current

@@ -74,12 +74,16 @@ def library() -> ctypes.CDLL:
             for name in ("pa_decode_mla", "pa_decode_mla_partition", "pa_decode_mla_merge"):
                 getattr(lib, name).argtypes = mla
                 getattr(lib, name).restype = ctypes.c_int
-            lib.pa_decode_kv_e4m3.argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp, f32, f32,
-                                              f32, vp, vp, sz, vp]
-            lib.pa_decode_kv_e4m3.restype = ctypes.c_int
-            lib.pa_decode_indexed.argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp,
-                                              ctypes.c_int, vp, f32, vp, vp, sz, vp]
-            lib.pa_decode_indexed.restype = ctypes.c_int
+            for name in ("pa_decode_kv_e4m3", "pa_decode_kv_e4m3_partition",
+                         "pa_decode_kv_e4m3_merge"):
+                getattr(lib, name).argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp, f32, f32,
+                                               f32, vp, vp, sz, vp]
+                getattr(lib, name).restype = ctypes.c_int
+            for name in ("pa_decode_indexed", "pa_decode_indexed_partition",
+                         "pa_decode_indexed_merge"):
+                getattr(lib, name).argtypes = [ctypes.POINTER(PADesc), vp, vp, vp, vp, vp,
+                                               ctypes.c_int, vp, f32, vp, vp, sz, vp]
+                getattr(lib, name).restype = ctypes.c_int
             lib.pa_workspace_size.argtypes = [ctypes.POINTER(PADesc)]
             lib.pa_workspace_size.restype = sz
             lib.pa_mla_workspace_size.argtypes = [ctypes.POINTER(PAMLADesc)]
@@ -212,13 +216,20 @@ def decode(q, k_cache, v_cache, block_table, context_lens, scale, out=None, work
     return out
 
 
+_KV8_PASSES = {"both": "pa_decode_kv_e4m3", "partition": "pa_decode_kv_e4m3_partition",
+               "merge": "pa_decode_kv_e4m3_merge"}
+_IDX_PASSES = {"both": "pa_decode_indexed", "partition": "pa_decode_indexed_partition",
+               "merge": "pa_decode_indexed_merge"}
+
+
 def decode_kv8(q, k_cache, v_cache, block_table, context_lens, scale, k_scale, v_scale,
-               out=None, workspace=None, num_partitions=0, stream=None):
+               out=None, workspace=None, num_partitions=0, stream=None, passes="both"):
     """pa_decode_kv_e4m3: paged GQA/MHA/MQA decode over a float8 KV cache.
 
     k_cache, v_cache [num_blocks, Hkv, block_size, 128] uint8 holding E4M3 codes;
     the key is code * k_scale and the value code * v_scale.  q [B, Hq, 128] fp16 or
     bf16 (bf16 within the fp16 range).  Returns out [B, Hq, 128] in q's dtype.
+    passes="partition" / "merge" run one of the two kernels, as for decode().
     """
     _require(q, "q", ndim=3)
     _require(k_cache, "k_cache", torch.uint8, 4)
@@ -243,20 +254,21 @@ def decode_kv8(q, k_cache, v_cache, block_table, context_lens, scale, k_scale, v
     if ws_bytes == 0:
         raise PAError(PA_ERR_UNSUPPORTED, "pa_workspace_size")
     ws = _workspace(ws_bytes, q.device, workspace)
-    _check(library().pa_decode_kv_e4m3(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                       _ptr(block_table), _ptr(context_lens), float(scale),
-                                       float(k_scale), float(v_scale), _ptr(out), _ptr(ws),
-                                       ws.numel() * ws.element_size(), _stream_ptr(stream)),
-           "pa_decode_kv_e4m3")
+    fn = _KV8_PASSES[passes]
+    _check(getattr(library(), fn)(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(block_table), _ptr(context_lens), float(scale),
+                                  float(k_scale), float(v_scale), _ptr(out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream_ptr(stream)), fn)
     return out
 
 
 def decode_indexed(q, k_cache, v_cache, block_table, token_index, n_sel, scale, out=None,
-                   workspace=None, num_partitions=0, stream=None):
+                   workspace=None, num_partitions=0, stream=None, passes="both"):
     """pa_decode_indexed: each sequence attends over a list of its token positions.
 
     token_index [B, max_sel] int32 positions; n_sel [B] int32 counts (entries past
     n_sel[b] are never read).  Caches and q as decode() (head_dim 128).
+    passes="partition" / "merge" run one of the two kernels, as for decode().
     """
     _require(q, "q", ndim=3)
     _require(k_cache, "k_cache", q.dtype, 4)
@@ -275,11 +287,12 @@ def decode_indexed(q, k_cache, v_cache, block_table, token_index, n_sel, scale, 
     if ws_bytes == 0:
         raise PAError(PA_ERR_UNSUPPORTED, "pa_workspace_size")
     ws = _workspace(ws_bytes, q.device, workspace)
-    _check(library().pa_decode_indexed(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                       _ptr(block_table), _ptr(token_index),
-                                       int(token_index.shape[1]), _ptr(n_sel), float(scale),
-                                       _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
-                                       _stream_ptr(stream)), "pa_decode_indexed")
+    fn = _IDX_PASSES[passes]
+    _check(getattr(library(), fn)(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(block_table), _ptr(token_index),
+                                  int(token_index.shape[1]), _ptr(n_sel), float(scale),
+                                  _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream_ptr(stream)), fn)
     return out
 
 

@@ -575,12 +575,48 @@ pa_status pa_decode_kv_e4m3(const pa_desc *desc, const void *q, const void *k_ca
                  workspace, workspace_bytes, stream, kModeKv8, k_scale, v_scale);
 }
 
+pa_status pa_decode_kv_e4m3_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *context_lens, float scale, float k_scale,
+                            float v_scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kPartition, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream, kModeKv8, k_scale, v_scale);
+}
+
+pa_status pa_decode_kv_e4m3_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *context_lens, float scale, float k_scale,
+                            float v_scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kMerge, desc, q, k_cache, v_cache, block_table, context_lens, scale, out,
+                 workspace, workspace_bytes, stream, kModeKv8, k_scale, v_scale);
+}
+
 pa_status pa_decode_indexed(const pa_desc *desc, const void *q, const void *k_cache,
                             const void *v_cache, const int32_t *block_table,
                             const int32_t *token_index, int max_sel, const int32_t *n_sel,
                             float scale, void *out, void *workspace, size_t workspace_bytes,
                             void *stream) {
   return run_gqa(kBoth, desc, q, k_cache, v_cache, block_table, n_sel, scale, out, workspace,
+                 workspace_bytes, stream, kModeIndexed, 1.f, 1.f, token_index, max_sel);
+}
+
+pa_status pa_decode_indexed_partition(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *token_index, int max_sel, const int32_t *n_sel,
+                            float scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kPartition, desc, q, k_cache, v_cache, block_table, n_sel, scale, out, workspace,
+                 workspace_bytes, stream, kModeIndexed, 1.f, 1.f, token_index, max_sel);
+}
+
+pa_status pa_decode_indexed_merge(const pa_desc *desc, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table,
+                            const int32_t *token_index, int max_sel, const int32_t *n_sel,
+                            float scale, void *out, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  return run_gqa(kMerge, desc, q, k_cache, v_cache, block_table, n_sel, scale, out, workspace,
                  workspace_bytes, stream, kModeIndexed, 1.f, 1.f, token_index, max_sel);
 }
 

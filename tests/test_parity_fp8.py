@@ -135,3 +135,19 @@ def test_subnormal_codes_are_exact(cuda_device):
     for parts in (0, 5):
         assert_close(run(d, inp, k_scale=128.0, v_scale=128.0, num_partitions=parts), ref,
                      f"subnormal parts={parts}")
+
+
+def test_partition_then_merge_equals_full_call(cuda_device):
+    inp = workloads.make(kv8(5, 32, 8, 16, (100, 1000, 2049, 7, 333), seed=13))
+    d = to_dev(inp, cuda_device)
+    args = (d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["context_lens"], inp["scale"],
+            inp["k_scale"], inp["v_scale"])
+    full = pa().decode_kv8(*args, num_partitions=37)
+    desc = pa().gqa_desc(d["q"], d["k_cache"], d["block_table"], 37)
+    ws = torch.full((pa().workspace_size(desc),), 0xAB, dtype=torch.uint8, device=cuda_device)
+    out = torch.empty_like(d["q"])
+    for passes in ("partition", "merge"):
+        pa().decode_kv8(*args, out=out, workspace=ws, num_partitions=37, passes=passes)
+    torch.cuda.synchronize()
+    assert pa().device_status() == 0
+    assert torch.equal(out, full)

@@ -116,3 +116,19 @@ def test_full_size_topk_sampled(cuda_device):
     hs = torch.randint(0, w.num_q_heads, (40,), generator=g).tolist()
     pairs = np.array(list(zip(bs_, hs)), np.int32)
     assert_close(out[pairs[:, 0], pairs[:, 1]], ref_of(inp, pairs=pairs), "topk full")
+
+
+def test_partition_then_merge_equals_full_call(cuda_device):
+    inp = workloads.make_indexed(small(B=4, ctx=900, top=80, seed=14))
+    d = to_dev(inp, cuda_device)
+    args = (d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["token_index"], d["n_sel"],
+            inp["scale"])
+    full = pa().decode_indexed(*args, num_partitions=29)
+    desc = pa().gqa_desc(d["q"], d["k_cache"], d["block_table"], 29)
+    ws = torch.full((pa().workspace_size(desc),), 0xAB, dtype=torch.uint8, device=cuda_device)
+    out = torch.empty_like(d["q"])
+    for passes in ("partition", "merge"):
+        pa().decode_indexed(*args, out=out, workspace=ws, num_partitions=29, passes=passes)
+    torch.cuda.synchronize()
+    assert pa().device_status() == 0
+    assert torch.equal(out, full)
