@@ -22,6 +22,10 @@ namespace {
 
 constexpr int kMaxBatch = 4096;            // prefix table lives in shared memory
 constexpr int kMaxBatchMla = 32768;        // the merge's prefix table: 128 KB of shared memory
+// Empty units at the start of every non-empty segment of a GQA stream: the
+// per-segment cost (query switch, partial or output rows, the first tile's
+// wait) in tiles, so that equal pieces take equal time on mixed lengths.
+constexpr int kSegUnits = 2;
 constexpr int kMaxPartitions = 1 << 20;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -401,6 +405,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     p.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
     p.seg_ctr = reinterpret_cast<unsigned long long *>(w + pl.off_ctr);
+    p.seg_units = mode == kModeIndexed ? 0 : kSegUnits;
     p.epoch = mode == kModeFused ? next_epoch() : 0u;
     cudaError_t err = cudaSuccess;
     if (!dispatch_gqa<LaunchPartition>(D, pl.NT, bf16, mode, pl.parts, st, maps, &p, &err))
@@ -414,6 +419,7 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     mp.lens = cl;
     mp.cap = mode == kModeIndexed ? max_sel : d->max_blocks_per_seq * d->block_size;
     mp.tile = pa::kTile;
+    mp.seg_units = mode == kModeIndexed ? 0 : kSegUnits;
     mp.out = out;
     mp.B = d->batch;
     mp.Hq = d->num_q_heads;
@@ -533,6 +539,7 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     mp.lens = cl;
     mp.cap = d->max_blocks_per_seq * d->block_size;
     mp.tile = pa::kMlaTile;
+    mp.seg_units = 0;
     mp.out = out;
     mp.B = d->batch;
     mp.Hq = pa::kMlaHeads;

@@ -233,10 +233,17 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows) {
 
 __device__ __forceinline__ int clamp_ctx(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
 
-// prefix[0] = 0, prefix[b + 1] = sum_{b' <= b} ceil(clamp(ctx[b']) / tile).  All threads.
+// Work units of a sequence of c tokens: its tiles, plus `extra` units standing
+// for the fixed cost of a segment (none for an empty sequence).
+__device__ __forceinline__ int seq_units(int c, int cap, int tile, int extra) {
+  const int P = (clamp_ctx(c, cap) + tile - 1) / tile;
+  return P > 0 ? P + extra : 0;
+}
+
+// prefix[0] = 0, prefix[b + 1] = sum_{b' <= b} seq_units(ctx[b']).  All threads.
 template <int NTHREADS>
 __device__ void tiles_prefix(const int32_t *ctx, int B, int cap, int tile, int *prefix,
-                             int *scratch, bool report) {
+                             int *scratch, bool report, int extra = 0) {
   const int per = (B + NTHREADS - 1) / NTHREADS;
   const int b0 = threadIdx.x * per;
   const int b1 = min(B, b0 + per);
@@ -244,7 +251,7 @@ __device__ void tiles_prefix(const int32_t *ctx, int B, int cap, int tile, int *
   for (int b = b0; b < b1; ++b) {
     const int c = ctx[b];
     if (report && (c < 0 || c > cap)) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
-    local += (clamp_ctx(c, cap) + tile - 1) / tile;
+    local += seq_units(c, cap, tile, extra);
   }
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int v = local;
@@ -259,7 +266,7 @@ __device__ void tiles_prefix(const int32_t *ctx, int B, int cap, int tile, int *
   for (int i = 0; i < w; ++i) run += scratch[i];
   if (threadIdx.x == 0) prefix[0] = 0;
   for (int b = b0; b < b1; ++b) {
-    run += (clamp_ctx(ctx[b], cap) + tile - 1) / tile;
+    run += seq_units(ctx[b], cap, tile, extra);
     prefix[b + 1] = run;
   }
   __syncthreads();

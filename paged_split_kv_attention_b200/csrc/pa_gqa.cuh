@@ -81,6 +81,9 @@ struct GqaParams {
   // single-pass merge: nonzero epoch = the last piece of a split segment merges it
   unsigned long long *seg_ctr;  // [B * Hkv] arrival counters (epoch << 32 | count)
   uint32_t epoch;
+  // Each non-empty segment's run of the flattened stream starts with seg_units
+  // empty units, so that pieces are cut by tiles plus a fixed cost per segment
+  int seg_units;
 };
 
 // MODE 0, 2 and 3: 16-bit rows in 128-byte swizzled slabs (2: gathered row by
@@ -117,11 +120,14 @@ __device__ __forceinline__ void locate_tile(const int *prefix, int B, int Hkv, l
   j = static_cast<int>(r - static_cast<long long>(kvh) * P);
 }
 
-// Cache row of the first token of flattened tile t, or -1 if its block id is
-// outside [0, nb) (recorded, never dereferenced).
+// Cache row of the first token of the tile at flattened unit t, -2 for one of a
+// segment's leading empty units, or -1 if its block id is outside [0, nb)
+// (recorded, never dereferenced).
 __device__ __forceinline__ int tile_row(const GqaParams &p, const int *prefix, long long t) {
   int b, kvh, j;
   locate_tile(prefix, p.B, p.Hkv, t, b, kvh, j);
+  j -= p.seg_units;
+  if (j < 0) return -2;
   const int jb = j / p.tiles_per_block;
   const int blk = __ldg(&p.block_table[static_cast<long long>(b) * p.mbs + jb]);
   if (blk < 0 || blk >= p.nb) return -1;
@@ -253,7 +259,8 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     for (long long off = (lo & ~127ll) + tid * 128ll; off < hi; off += kGqaThreads * 128ll)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + off));
   }
-  tiles_prefix<kGqaThreads>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0);
+  tiles_prefix<kGqaThreads>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0,
+                            p.seg_units);
   // let the merge grid be scheduled as SMs free up (it waits for this grid to finish)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // sequences with no tokens get an all-zero output row (spread over the grid)
@@ -354,8 +361,8 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     const long long n = issued - wb;
     const int st = static_cast<int>(n % R);
     if (lane == 0) {
-      if (row < 0) {
-        record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
+      if (row < 0) {                                  // bad block id, or an empty unit
+        if (row == -1) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
         stage_valid[st] = 0;
         mbar_arrive(&full[st]);
       } else {
@@ -474,11 +481,16 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
 
   long long t = wb;
   while (t < we) {
-    const int P = prefix[b + 1] - prefix[b];
+    const int U = prefix[b + 1] - prefix[b];       // units of the segment
+    const int P = U - p.seg_units;                 // its tiles
     const long long seg_first = static_cast<long long>(p.Hkv) * prefix[b] +
-                                static_cast<long long>(kvh) * P;
-    const long long seg_end = min(we, seg_first + P);
-    const bool whole = seg_first >= wb && seg_first + P <= we;
+                                static_cast<long long>(kvh) * U;
+    const long long tile_first = seg_first + p.seg_units;
+    const long long seg_end = min(we, seg_first + U);
+    // whole: every tile of the segment is in this piece (its output is written
+    // here); has_tiles: this piece holds at least one of them
+    const bool whole = tile_first >= wb && seg_first + U <= we;
+    const bool has_tiles = seg_end > max(t, tile_first);
     // prefetch the next segment's query fragments and length
     int nb_ = b, nkvh = kvh, nj, nctx = ctx;
     if (seg_end < we) {
@@ -514,7 +526,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                abort_flag));
         if (!ok_cur) aborted = true;
       }
-      const int jt = static_cast<int>(t - seg_first);
+      const int jt = static_cast<int>(t - tile_first);
       const int ntok = (ok_cur && stage_valid[st]) ? min(kTile, ctx - jt * kTile) : 0;
       const uint32_t kb = ring_base + st * L::kStage;
       if (ntok > 0) {
@@ -636,30 +648,32 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     const long long slot = gw + seg;
     uint16_t *orow = reinterpret_cast<uint16_t *>(p.out) +
                      (static_cast<long long>(b) * p.Hq + kvh * p.G) * D;
+    if (has_tiles) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int h = nt * 8 + 2 * tq + e;
-        if (h >= p.G) continue;
-        const float inv = l[nt][e] > 0.f ? p.v_scale / l[nt][e] : 0.f;
+        for (int e = 0; e < 2; ++e) {
+          const int h = nt * 8 + 2 * tq + e;
+          if (h >= p.G) continue;
+          const float inv = l[nt][e] > 0.f ? p.v_scale / l[nt][e] : 0.f;
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt)
+          for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int d = KV8 ? mt * 16 + 2 * g + hf : mt * 16 + g + hf * 8;
-            const float val = o[mt][nt][hf * 2 + e] * inv;
-            if (whole) orow[h * D + d] = to16<BF16>(val);
-            else p.part_o[(slot * p.G + h) * D + d] = val;
-          }
-        if (!whole && g == 0)
-          p.part_lse[slot * p.G + h] = l[nt][e] > 0.f ? m[nt][e] + log2f(l[nt][e]) : -INFINITY;
-      }
+            for (int hf = 0; hf < 2; ++hf) {
+              const int d = KV8 ? mt * 16 + 2 * g + hf : mt * 16 + g + hf * 8;
+              const float val = o[mt][nt][hf * 2 + e] * inv;
+              if (whole) orow[h * D + d] = to16<BF16>(val);
+              else p.part_o[(slot * p.G + h) * D + d] = val;
+            }
+          if (!whole && g == 0)
+            p.part_lse[slot * p.G + h] = l[nt][e] > 0.f ? m[nt][e] + log2f(l[nt][e]) : -INFINITY;
+        }
+    }
     // single-pass merge: only a piece's first and last segments can be split;
     // their arrivals wait until the piece is done, off the streaming path
-    if (FUSED && !whole && n_split < 2) {
+    if (FUSED && !whole && has_tiles && n_split < 2) {
       split_seg[n_split] = seg;
-      split_first[n_split] = seg_first;
+      split_first[n_split] = tile_first;
       split_tiles[n_split] = P;
       ++n_split;
     }

@@ -31,6 +31,7 @@ struct MergeParams {
   const float *part_lse;     // [slots][G]
   const int32_t *lens;       // [B] the partition pass's sequence lengths (tokens)
   int cap, tile;             // its length clamp and tokens per tile
+  int seg_units;             // leading units of a segment that hold no tile
   void *out;                 // [B][Hq][DV] 16-bit
   int B, Hq, Hkv, G;
   int pieces;                // pieces launched by the partition pass
@@ -57,15 +58,17 @@ merge_kernel(const MergeParams p) {
   extern __shared__ int merge_prefix[];      // [B + 1], then 8 ints of scan scratch
 
   tiles_prefix<kMergeThreads>(p.lens, p.B, p.cap, p.tile, merge_prefix,
-                              merge_prefix + p.B + 1, false);
+                              merge_prefix + p.B + 1, false, p.seg_units);
   const int *prefix = merge_prefix;
   const int seg = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int b = seg / p.Hkv, kvh = seg - (seg / p.Hkv) * p.Hkv;
-  const int P = prefix[b + 1] - prefix[b];
-  if (P <= 0 || h >= p.G) return;
+  const int U = prefix[b + 1] - prefix[b];       // the segment's units
+  if (U <= 0 || h >= p.G) return;
+  const int P = U - p.seg_units;                  // its tiles, after seg_units empty units
   const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
   const int pieces = used_pieces(p.pieces, TP, p.min_tiles, p.floor_pieces);
-  const long long first = static_cast<long long>(p.Hkv) * prefix[b] + static_cast<long long>(kvh) * P;
+  const long long first = static_cast<long long>(p.Hkv) * prefix[b] +
+                          static_cast<long long>(kvh) * U + p.seg_units;
   const int g0 = piece_of(first, TP, pieces);
   const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
@@ -139,7 +142,7 @@ merge_rows_kernel(const MergeParams p) {
   static_assert(V4 * 128 == DV, "DV must be a multiple of 128");
   extern __shared__ int merge_prefix[];          // [B + 1], then 8 ints of scan scratch
   tiles_prefix<kMergeRowsPerCta * 32>(p.lens, p.B, p.cap, p.tile, merge_prefix,
-                                      merge_prefix + p.B + 1, false);
+                                      merge_prefix + p.B + 1, false, p.seg_units);
   const int *prefix = merge_prefix;
   const int lane = threadIdx.x & 31;
   const long long r = static_cast<long long>(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
@@ -147,11 +150,13 @@ merge_rows_kernel(const MergeParams p) {
   if (r >= segs * p.G) return;
   const int seg = static_cast<int>(r / p.G), h = static_cast<int>(r - static_cast<long long>(seg) * p.G);
   const int b = seg / p.Hkv, kvh = seg - (seg / p.Hkv) * p.Hkv;
-  const int P = prefix[b + 1] - prefix[b];
-  if (P <= 0) return;
+  const int U = prefix[b + 1] - prefix[b];       // the segment's units
+  if (U <= 0) return;
+  const int P = U - p.seg_units;                  // its tiles, after seg_units empty units
   const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
   const int pieces = used_pieces(p.pieces, TP, p.min_tiles, p.floor_pieces);
-  const long long first = static_cast<long long>(p.Hkv) * prefix[b] + static_cast<long long>(kvh) * P;
+  const long long first = static_cast<long long>(p.Hkv) * prefix[b] +
+                          static_cast<long long>(kvh) * U + p.seg_units;
   const int g0 = piece_of(first, TP, pieces);
   const int g1 = piece_of(first + P - 1, TP, pieces);
   if (g0 == g1) return;
