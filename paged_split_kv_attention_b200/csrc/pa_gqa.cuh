@@ -11,30 +11,36 @@
 // (sequence, kv head) writes the final output directly.
 //
 // How the pieces are chosen.  The KV stream is flattened into 16-token tiles in
-// (sequence, kv head, tile) order and cut into P equal runs of tiles, one per
-// warp of a persistent grid (P = CTAs x 8 warps): every warp reads the same
-// number of bytes whatever the mix of context lengths.  Where a warp's run
-// crosses (sequence, kv head) boundaries -- a "segment" -- it produces one
-// result per segment it touches.  The split points therefore fall where the
-// work balances, not at a fixed length.
+// (sequence, kv head, tile) order, each non-empty (sequence, kv head) -- a
+// "segment" -- preceded by seg_units empty units that stand for its fixed cost
+// (query switch, output rows, the first tile's wait).  The stream is cut into P
+// equal runs of units, one per warp of a persistent grid (P = CTAs x 8 warps),
+// so every warp carries the same work whatever the mix of context lengths.  A
+// warp produces one result per segment whose tiles it touches.  The split
+// points therefore fall where the work balances, not at a fixed length.
 //
 // Merge.  A warp that ends a segment it shares with other warps writes its
 // normalised partial and log-sum-exp into slot (warp piece + segment); the merge
 // kernel (pa_merge.cuh), launched right behind this one with programmatic
 // dependent launch, combines them.  No barrier, fence or atomic is needed on
-// the streaming path.
+// the streaming path.  In the single-pass form (MODE 3) each piece counts itself
+// in at its split segments once its last tile is done, and the last to arrive
+// merges the segment.
 //
 // Data movement (the pages ask that K and V be loaded in parallel as fast as
 // possible, then rescaled and combined).  Each warp is its own pipeline: lane 0
 // issues TMA tensor copies (128-byte swizzle, L2 evict-first) of the next R
 // tiles' K and V (16 x D each, physical block looked up through the block table
 // by a 32-tile look-ahead held one tile per lane) into the warp's R-stage ring,
-// each stage guarded by an mbarrier.  Per tile the warp computes S^T = K Q^T with
-// mma.sync m16n8k16 (tokens on M, the group's heads on N), the online softmax in
-// registers (max over tokens with three xor shuffles, sums kept per lane) and
-// O^T += V^T P with V^T fragments from ldmatrix.trans and P moved to the B
-// operand layout with movmatrix (as a 16-bit hi + lo pair, two MMAs).  The query
-// fragments of the next segment are prefetched into registers.
+// each stage guarded by an mbarrier (at D 128 one 3-D box lands both 64-wide
+// slabs of a tile).  Per tile the warp computes S^T = K Q^T with mma.sync
+// m16n8k16 (tokens on M, the group's heads on N; two accumulators over the
+// k-steps), the online softmax in registers (max over tokens with three xor
+// shuffles, sums kept per lane) and O^T += V^T P with V^T fragments from
+// ldmatrix.trans and P moved to the B operand layout with movmatrix (as a 16-bit
+// hi + lo pair, two MMAs).  On the 16-bit TMA path the scores of tile t + 1 are
+// taken before tile t's softmax, so each iteration holds two independent MMA
+// chains.  The query fragments of the next segment are prefetched into registers.
 //
 // Float8 KV cache (KV8).  With E4M3 codes in the cache (one key scale and one
 // value scale per tensor; page "bjpcjp.github.io: llms-attention",
