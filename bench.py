@@ -21,6 +21,7 @@ the operation) on a bounded sample of the same workload on this host's cores.
 from __future__ import annotations
 
 import argparse
+import re
 import hashlib
 import json
 import math
@@ -206,10 +207,15 @@ def measured_peaks():
 
 
 def kernel_hash(files):
+    """Hash of the kernel sources with comments and blank space removed: traffic
+    counters stay valid across comment edits, and go stale on any code change."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "paged_split_kv_attention_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "paged_split_kv_attention_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 
