@@ -211,6 +211,8 @@ pa_status pa_decode_kv_e4m3_merge(const pa_desc *desc, const void *q, const void
  *   block_table[b][pos / block_size]); entries past n_sel[b] are never read, a
  *   position listed twice counts twice, the order does not matter.
  * n_sel: device int32 [batch], 0 <= n_sel[b] <= max_sel (0 = all-zero output).
+ * max_sel >= 1, with batch x (max_sel / 16 + 1) x num_kv_heads < 2^31
+ * (PA_ERR_UNSUPPORTED otherwise).
  * Everything else as pa_decode (16-bit q / caches / out, head_dim 128).  A
  * position outside [0, max_blocks_per_seq x block_size) or a block id outside
  * the pool is skipped and reported as PA_ERR_BAD_BLOCK_ID by pa_device_status.

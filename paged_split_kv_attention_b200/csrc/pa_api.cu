@@ -196,7 +196,8 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, int mode = kMode16) {
   const int64_t kv_rows = int64_t(d->num_blocks) * d->num_kv_heads * d->block_size;
   const int64_t q_rows = int64_t(d->batch) * d->num_q_heads;
   const int64_t cap = int64_t(d->max_blocks_per_seq) * d->block_size;
-  const int64_t max_tiles = int64_t(d->batch) * (cap / pa::kTile) * d->num_kv_heads;
+  // work units of the flattened stream: tiles plus kSegUnits per segment
+  const int64_t max_tiles = int64_t(d->batch) * (cap / pa::kTile + kSegUnits) * d->num_kv_heads;
   if (kv_rows > INT32_MAX || q_rows > INT32_MAX || cap > INT32_MAX || max_tiles > INT32_MAX)
     return PA_ERR_UNSUPPORTED;
   pl->G = G;
@@ -364,6 +365,10 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
   if (mode == kModeIndexed &&
       (!token_index || (reinterpret_cast<uintptr_t>(token_index) & 3u) || max_sel <= 0))
     return PA_ERR_INVALID_ARG;
+  // the index-list stream counts tiles of up to max_sel entries per sequence
+  if (mode == kModeIndexed &&
+      int64_t(d->batch) * (max_sel / pa::kTile + 1) * d->num_kv_heads > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
   const bool bf16 = d->dtype == PA_BF16;

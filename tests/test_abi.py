@@ -122,3 +122,14 @@ def test_fused_entry_point_rejects_what_pa_decode_rejects(lib):
         d = _desc(**bad)
         assert (lib.pa_decode_fused(ctypes.byref(d), z, z, z, z, z, 0.1, z, z, 1 << 30, None) ==
                 lib.pa_decode(ctypes.byref(d), z, z, z, z, z, 0.1, z, z, 1 << 30, None) != 0)
+
+
+def test_index_list_size_limit(lib):
+    import paged_split_kv_attention_b200 as pa
+    z = ctypes.c_void_p(0x1000)
+    d = _desc(batch=4096, num_kv_heads=8, num_q_heads=32)
+    huge = (1 << 31) // (4096 * 8) * 16
+    assert lib.pa_decode_indexed(ctypes.byref(d), z, z, z, z, z, huge, z, 0.1, z, z, 1 << 30,
+                                 None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_indexed(ctypes.byref(d), z, z, z, z, z, 0, z, 0.1, z, z, 1 << 30,
+                                 None) == pa.PA_ERR_INVALID_ARG
