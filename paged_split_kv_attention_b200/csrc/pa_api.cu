@@ -125,15 +125,17 @@ enum GqaMode { kMode16 = 0, kModeKv8 = 1, kModeIndexed = 2, kModeFused = 3 };
 
 template <int D, int NT, bool BF16, int MODE>
 struct GqaVariant {
-  // 24 KB ring per warp: 3 x 8 KB (D 128), 6 x 4 KB (D 64 or float8 D 128)
-  static constexpr int R = MODE == kModeKv8 ? 6 : (D == 128 ? 3 : 6);
-  using L = pa::GqaLayout<D, NT, R, MODE>;
+  // 192 KB of rings per CTA: 8 warps x 3 x 8 KB (D 128), 8 x 6 x 4 KB (D 64, or
+  // float8 at 16 heads per group), 12 x 4 x 4 KB (float8 up to 8 heads per group)
+  static constexpr int W = pa::gqa_warps(MODE, NT);
+  static constexpr int R = MODE == kModeKv8 ? (W == 12 ? 4 : 6) : (D == 128 ? 3 : 6);
+  using L = pa::GqaLayout<D, NT, R, MODE, W>;
   static const void *kernel() {
-    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, MODE>);
+    return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, MODE, W>);
   }
   static void launch(int grid, size_t smem, cudaStream_t st, const CUtensorMap &k,
                      const CUtensorMap &v, const pa::GqaParams &p) {
-    pa::gqa_decode_kernel<D, NT, BF16, R, MODE><<<grid, pa::kGqaThreads, smem, st>>>(k, v, p);
+    pa::gqa_decode_kernel<D, NT, BF16, R, MODE, W><<<grid, 32 * W, smem, st>>>(k, v, p);
   }
 };
 
@@ -162,12 +164,12 @@ template <int D, int NT, bool BF16, int MODE>
 struct QueryResident {
   static void run(int B, int *out) {
     using V = GqaVariant<D, NT, BF16, MODE>;
-    *out = resident_ctas(V::kernel(), pa::kGqaThreads, V::L::bytes(B));
+    *out = resident_ctas(V::kernel(), 32 * V::W, V::L::bytes(B));
   }
 };
 
 struct GqaPlan {
-  int G = 0, NT = 0, parts = 0;
+  int G = 0, NT = 0, parts = 0, warps = pa::kWarps;
   size_t off_lse = 0, off_o = 0, off_ctr = 0, bytes = 0;
 };
 
@@ -208,7 +210,8 @@ pa_status plan_gqa(const pa_desc *d, GqaPlan *pl, int mode = kMode16) {
     if (pl->parts <= 0) return PA_ERR_CUDA;
   }
   // one partial slot per (warp piece, segment) pair a piece can end: piece + segment
-  const size_t slots = size_t(pl->parts) * pa::kWarps + size_t(d->batch) * d->num_kv_heads;
+  pl->warps = pa::gqa_warps(mode, pl->NT);
+  const size_t slots = size_t(pl->parts) * pl->warps + size_t(d->batch) * d->num_kv_heads;
   pl->off_lse = 0;
   pl->off_o = pl->off_lse + round_up(slots * G * 4, 256);
   // arrival counters of the single-pass merge, one 64-bit word per segment
@@ -430,9 +433,9 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     mp.Hq = d->num_q_heads;
     mp.Hkv = d->num_kv_heads;
     mp.G = pl.G;
-    mp.pieces = pl.parts * pa::kWarps;
+    mp.pieces = pl.parts * pl.warps;
     mp.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
-    mp.floor_pieces = static_cast<long long>(pa::kWarps) * d->batch * d->num_kv_heads;
+    mp.floor_pieces = static_cast<long long>(pl.warps) * d->batch * d->num_kv_heads;
     if (merge_dispatch(D, bf16, mp, d->batch * d->num_kv_heads, st) != cudaSuccess)
       return PA_ERR_CUDA;
   }

@@ -14,7 +14,8 @@
 // (sequence, kv head, tile) order, each non-empty (sequence, kv head) -- a
 // "segment" -- preceded by seg_units empty units that stand for its fixed cost
 // (query switch, output rows, the first tile's wait).  The stream is cut into P
-// equal runs of units, one per warp of a persistent grid (P = CTAs x 8 warps),
+// equal runs of units, one per warp of a persistent grid (P = CTAs x 8 warps;
+// 12 in the float8 mode at up to 8 heads per group),
 // so every warp carries the same work whatever the mix of context lengths.  A
 // warp produces one result per segment whose tiles it touches.  The split
 // points therefore fall where the work balances, not at a fixed length.
@@ -63,8 +64,15 @@
 namespace pa {
 
 constexpr int kTile = 16;               // tokens per pipeline tile
-constexpr int kWarps = 8;               // independent streaming warps per CTA
+constexpr int kWarps = 8;               // independent streaming warps per CTA (default)
 constexpr int kGqaThreads = 32 * kWarps;
+
+// Warps per CTA of a kernel variant: the float8 mode at up to 8 heads per group
+// runs 12 (its 4 KB tiles leave each warp latency-bound, and 12 x 4 stages of
+// 4 KB fill the same shared memory as 8 x 6); every other variant runs 8.
+__host__ __device__ constexpr int gqa_warps(int mode, int nt) {
+  return mode == 1 && nt == 1 ? 12 : kWarps;
+}
 
 struct GqaParams {
   const uint16_t *q;            // [B][Hq][D]
@@ -94,15 +102,15 @@ struct GqaParams {
 
 // MODE 0, 2 and 3: 16-bit rows in 128-byte swizzled slabs (2: gathered row by
 // row into the same layout).  MODE 1: float8 rows.
-template <int D, int NT, int R, int MODE = 0>
+template <int D, int NT, int R, int MODE = 0, int W = kWarps>
 struct GqaLayout {
   static constexpr int kHeads = 8 * NT;            // group width padded to the MMA N
   static constexpr int kKTile = kTile * D * (MODE == 1 ? 1 : 2);  // bytes of one K (or V) tile
   static constexpr int kStage = 2 * kKTile;
   static constexpr int ring = 0;                   // warp w: stages [w*R, (w+1)*R)
-  static constexpr int bars = ring + kWarps * R * kStage;
-  static constexpr int nbars = kWarps * R;
-  static constexpr int info = bars + nbars * 8;     // int stage_valid[kWarps * R]
+  static constexpr int bars = ring + W * R * kStage;
+  static constexpr int nbars = W * R;
+  static constexpr int info = bars + nbars * 8;     // int stage_valid[W * R]
   static constexpr int flags = info + nbars * 4;    // abort flag + scan scratch
   static constexpr int prefix = flags + 64;         // int prefix[B + 1]
   static size_t bytes(int B) { return 1024 + prefix + static_cast<size_t>(B + 1) * 4; }
@@ -232,15 +240,17 @@ __device__ __forceinline__ void load_q(const GqaParams &p, int b, int kvh, int l
 // MODE 0: 16-bit cache, TMA tiles.  1: float8 cache (KV8).  2: index-list
 // decode (IDX): each warp gathers its tiles' selected rows with cp.async.
 // 3: as 0, and the last piece of each split segment merges it (FUSED).
-template <int D, int NT, bool BF16, int R, int MODE = 0>
-__global__ void __launch_bounds__(kGqaThreads, 1)
+template <int D, int NT, bool BF16, int R, int MODE = 0, int W = kWarps>
+__global__ void __launch_bounds__(32 * W, 1)
 gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const GqaParams p) {
   constexpr bool KV8 = MODE == 1, IDX = MODE == 2, FUSED = MODE == 3;
   // 16-bit TMA modes: the next tile's scores are taken ahead of this tile's
   // softmax (measured slower for the float8 and index-list modes)
   constexpr bool PIPE = !KV8 && !IDX;
-  using L = GqaLayout<D, NT, R, MODE>;
+  using L = GqaLayout<D, NT, R, MODE, W>;
+  constexpr int kThreadsW = 32 * W;
+  static_assert(W <= 12, "the scan scratch in the flags area holds 12 warps");
   static_assert(!KV8 || D == 128, "the float8 KV path reads 128-byte rows");
   static_assert(!IDX || D == 128, "index-list gathers read 256-byte rows");
   constexpr bool CT = BF16 && !KV8;          // MMA operand type: bf16, else fp16
@@ -262,23 +272,23 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     const char *tb = reinterpret_cast<const char *>(p.block_table);
     const long long bytes = static_cast<long long>(p.B) * p.mbs * 4;
     const long long lo = bytes * c / p.parts, hi = bytes * (c + 1) / p.parts;
-    for (long long off = (lo & ~127ll) + tid * 128ll; off < hi; off += kGqaThreads * 128ll)
+    for (long long off = (lo & ~127ll) + tid * 128ll; off < hi; off += kThreadsW * 128ll)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + off));
   }
-  tiles_prefix<kGqaThreads>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0,
+  tiles_prefix<kThreadsW>(p.context_lens, p.B, cap, kTile, prefix, scan_scratch, c == 0,
                             p.seg_units);
   // let the merge grid be scheduled as SMs free up (it waits for this grid to finish)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // sequences with no tokens get an all-zero output row (spread over the grid)
   for (int b = c; b < p.B; b += p.parts)
     if (prefix[b + 1] == prefix[b])
-      for (int i = tid; i < p.Hq * D; i += kGqaThreads)
+      for (int i = tid; i < p.Hq * D; i += kThreadsW)
         reinterpret_cast<uint16_t *>(p.out)[static_cast<long long>(b) * p.Hq * D + i] = 0;
 
   const long long TP = static_cast<long long>(p.Hkv) * prefix[p.B];
-  const int pieces = used_pieces(p.parts * kWarps, TP, p.min_tiles,
-                                 static_cast<long long>(kWarps) * p.B * p.Hkv);
-  const int gw = c * kWarps + warp;                     // this warp's piece
+  const int pieces = used_pieces(p.parts * W, TP, p.min_tiles,
+                                 static_cast<long long>(W) * p.B * p.Hkv);
+  const int gw = c * W + warp;                     // this warp's piece
   const long long wb = gw < pieces ? piece_begin(gw, TP, pieces) : 0;
   const long long we = gw < pieces ? piece_begin(gw + 1, TP, pieces) : 0;
 
