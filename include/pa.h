@@ -78,8 +78,8 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
  * Supported: head_dim in {64, 128}; block_size a multiple of 16 up to 1024;
  * 1 <= num_q_heads / num_kv_heads <= 16; 0 <= batch <= 4096 (0 is a no-op).
  * num_partitions: CTAs of the partition grid; the flattened KV stream is cut into
- * equal-work pieces, one per warp: 8 per CTA (12 in pa_decode_kv_e4m3 at up to 8
- * query heads per kv head).  0 picks (SM count) x (resident CTAs
+ * equal-work pieces, one per warp: 8 per CTA (12 in pa_decode_kv_e4m3 and
+ * pa_decode_indexed at up to 8 query heads per kv head).  0 picks (SM count) x (resident CTAs
  * per SM) for the current device, with pieces no shorter than the partial output
  * they write. */
 typedef struct {
@@ -237,7 +237,8 @@ pa_status pa_decode_indexed_merge(const pa_desc *desc, const void *q, const void
                                   size_t workspace_bytes, void *stream);
 
 /* Number of partitions (CTAs of the partition pass; each runs 8 independently
- * streaming warps, one piece each, 12 for the float8 path at up to 8 heads per group) a call with num_partitions == 0 uses on the current
+ * streaming warps, one piece each; 12 for the float8 and index-list paths at up to 8
+ * heads per group) a call with num_partitions == 0 uses on the current
  * device (SM count x resident CTAs per SM), or -1 without a usable device.
  * kind: 0 = GQA with this head_dim, 1 = MLA (head_dim ignored), 2 = GQA over a
  * float8 KV cache (head_dim 128), 3 = index-list decode (head_dim 128). */

@@ -126,9 +126,12 @@ enum GqaMode { kMode16 = 0, kModeKv8 = 1, kModeIndexed = 2, kModeFused = 3 };
 template <int D, int NT, bool BF16, int MODE>
 struct GqaVariant {
   // 192 KB of rings per CTA: 8 warps x 3 x 8 KB (D 128), 8 x 6 x 4 KB (D 64, or
-  // float8 at 16 heads per group), 12 x 4 x 4 KB (float8 up to 8 heads per group)
+  // float8 at 16 heads per group), 12 x 4 x 4 KB (float8 up to 8 heads per group),
+  // 12 x 2 x 8 KB (index list up to 8 heads per group)
   static constexpr int W = pa::gqa_warps(MODE, NT);
-  static constexpr int R = MODE == kModeKv8 ? (W == 12 ? 4 : 6) : (D == 128 ? 3 : 6);
+  static constexpr int R = MODE == kModeKv8       ? (W == 12 ? 4 : 6)
+                           : MODE == kModeIndexed ? (W == 12 ? 2 : 3)
+                                                  : (D == 128 ? 3 : 6);
   using L = pa::GqaLayout<D, NT, R, MODE, W>;
   static const void *kernel() {
     return reinterpret_cast<const void *>(&pa::gqa_decode_kernel<D, NT, BF16, R, MODE, W>);

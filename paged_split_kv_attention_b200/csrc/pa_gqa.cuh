@@ -15,7 +15,7 @@
 // "segment" -- preceded by seg_units empty units that stand for its fixed cost
 // (query switch, output rows, the first tile's wait).  The stream is cut into P
 // equal runs of units, one per warp of a persistent grid (P = CTAs x 8 warps;
-// 12 in the float8 mode at up to 8 heads per group),
+// 12 in the float8 and index-list modes at up to 8 heads per group),
 // so every warp carries the same work whatever the mix of context lengths.  A
 // warp produces one result per segment whose tiles it touches.  The split
 // points therefore fall where the work balances, not at a fixed length.
@@ -67,11 +67,13 @@ constexpr int kTile = 16;               // tokens per pipeline tile
 constexpr int kWarps = 8;               // independent streaming warps per CTA (default)
 constexpr int kGqaThreads = 32 * kWarps;
 
-// Warps per CTA of a kernel variant: the float8 mode at up to 8 heads per group
-// runs 12 (its 4 KB tiles leave each warp latency-bound, and 12 x 4 stages of
-// 4 KB fill the same shared memory as 8 x 6); every other variant runs 8.
+// Warps per CTA of a kernel variant.  The float8 (1) and index-list (2) modes at
+// up to 8 heads per group run 12: each of their warps is latency-bound (widening
+// the codes; the lookup chain and row gathers), and 12 x 4 stages of 4 KB, or
+// 12 x 2 stages of 8 KB, fill the same shared memory as 8 warps do.  Every other
+// variant runs 8.
 __host__ __device__ constexpr int gqa_warps(int mode, int nt) {
-  return mode == 1 && nt == 1 ? 12 : kWarps;
+  return (mode == 1 || mode == 2) && nt == 1 ? 12 : kWarps;
 }
 
 struct GqaParams {
