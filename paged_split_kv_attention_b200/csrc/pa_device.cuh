@@ -231,11 +231,11 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows) {
                                ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
 
-__device__ __forceinline__ int clamp_ctx(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
+__host__ __device__ __forceinline__ int clamp_ctx(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
 
 // Work units of a sequence of c tokens: its tiles, plus `extra` units standing
 // for the fixed cost of a segment (none for an empty sequence).
-__device__ __forceinline__ int seq_units(int c, int cap, int tile, int extra) {
+__host__ __device__ __forceinline__ int seq_units(int c, int cap, int tile, int extra) {
   const int P = (clamp_ctx(c, cap) + tile - 1) / tile;
   return P > 0 ? P + extra : 0;
 }
@@ -274,18 +274,18 @@ __device__ void tiles_prefix(const int32_t *ctx, int B, int cap, int tile, int *
 
 // Partition of a flattened work stream of `total` units into `parts` equal
 // pieces: piece c covers [begin(c), begin(c + 1)).
-__device__ __forceinline__ long long piece_begin(long long c, long long total, long long parts) {
+__host__ __device__ __forceinline__ long long piece_begin(long long c, long long total, long long parts) {
   return (c * total) / parts;
 }
 
 // Pieces actually used out of `parts` launched.  With min_units > 0 (an
-// automatic launch) a short stream is not cut finer than min_units per piece,
-// so that partial outputs and their merge stay small next to the work itself,
-// but into at least floor_pieces pieces, so that a short stream still spreads
-// over several warps; with min_units == 0 (an explicit partition count) every
-// piece is used.  The partition and merge kernels compute it from the same
-// arguments.
-__device__ __forceinline__ int used_pieces(int parts, long long total, int min_units,
+// automatic launch) a short stream is cut into the fewest pieces of at most
+// min_units units each (so pieces stay near min_units and the partial outputs
+// and their merge stay small next to the work itself), but into at least
+// floor_pieces pieces, so that a short stream still spreads over several warps;
+// with min_units == 0 (an explicit partition count) every piece is used.  The
+// partition and merge kernels compute it from the same arguments.
+__host__ __device__ __forceinline__ int used_pieces(int parts, long long total, int min_units,
                                            long long floor_pieces) {
   if (min_units <= 0) return parts;
   long long want = (total + min_units - 1) / min_units;
@@ -294,7 +294,7 @@ __device__ __forceinline__ int used_pieces(int parts, long long total, int min_u
 }
 
 // The piece that owns unit t (0 <= t < total).
-__device__ __forceinline__ int piece_of(long long t, long long total, long long parts) {
+__host__ __device__ __forceinline__ int piece_of(long long t, long long total, long long parts) {
   return static_cast<int>(((t + 1) * parts + total - 1) / total - 1);
 }
 
