@@ -462,7 +462,7 @@ def run_ours(args, rank, world, local):
                 "peak_source": f"{peak_src} hbm_gbs (copy)",
                 "nominal_frac_8tbs": round(achieved / 8000.0, 4)}
     if w.kind == "mla":
-        # a dense contraction (~240 flop per latent byte): judged against the
+        # a dense contraction (~240 flop per latent byte): measured against the
         # tensor roofline; the step loop runs for seconds, so the sustained peak
         fl = workloads.flops(w, inp["context_lens"])
         tflops = fl / part_avg_s / 1e12
