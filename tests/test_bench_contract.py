@@ -1,0 +1,52 @@
+"""CPU checks of bench.py's output contract on its reference arm (the float64
+oracle timed on host cores): one JSON line with the required keys, alone and
+under torchrun with two ranks, where rank 0 alone prints."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+REQUIRED = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+            "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "impl",
+            "cpu_baseline", "e2e")
+
+
+def json_lines(out):
+    return [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+
+
+def check_line(j, n_gpus):
+    for k in REQUIRED:
+        assert k in j, k
+    assert j["impl"] == "reference" and j["n_gpus"] == n_gpus and j["steps"] == 2
+    assert j["value"] > 0 and j["higher_is_better"] is True and j["dtype"] == "f64"
+    assert "workload" in j["config"]
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == j["value"]
+    e = j["e2e"]
+    assert e["value"] == j["value"] and e["unit"] == j["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
+                        "--warmup", "3", "--workload", "tiny"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = json_lines(r.stdout)
+    assert len(lines) == 1
+    check_line(lines[0], 1)
+
+
+def test_reference_arm_under_two_ranks():
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", "29541", "bench.py", "--impl", "reference", "--gpus", "2",
+                        "--steps", "2", "--warmup", "3", "--workload", "tiny"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = json_lines(r.stdout)
+    assert len(lines) == 1                   # rank 0 alone prints
+    check_line(lines[0], 2)
