@@ -133,3 +133,24 @@ def test_index_list_size_limit(lib):
                                  None) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_indexed(ctypes.byref(d), z, z, z, z, z, 0, z, 0.1, z, z, 1 << 30,
                                  None) == pa.PA_ERR_INVALID_ARG
+
+
+def test_float8_entry_point_validation(lib):
+    import paged_split_kv_attention_b200 as pa
+    z = ctypes.c_void_p(0x1000)
+    d = _desc()
+    for ks, vs in ((float("nan"), 1.0), (1.0, float("inf")), (float("-inf"), 1.0)):
+        assert lib.pa_decode_kv_e4m3(ctypes.byref(d), z, z, z, z, z, 0.1, ks, vs, z, z, 1 << 30,
+                                     None) == pa.PA_ERR_INVALID_ARG
+    d64 = _desc(head_dim=64)
+    assert lib.pa_decode_kv_e4m3(ctypes.byref(d64), z, z, z, z, z, 0.1, 1.0, 1.0, z, z, 1 << 30,
+                                 None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_indexed(ctypes.byref(d64), z, z, z, z, z, 16, z, 0.1, z, z, 1 << 30,
+                                 None) == pa.PA_ERR_UNSUPPORTED
+    # the partition / merge forms validate alike
+    for name in ("pa_decode_kv_e4m3_partition", "pa_decode_kv_e4m3_merge"):
+        assert getattr(lib, name)(ctypes.byref(d), z, z, z, z, z, 0.1, float("nan"), 1.0, z, z,
+                                  1 << 30, None) == pa.PA_ERR_INVALID_ARG
+    for name in ("pa_decode_indexed_partition", "pa_decode_indexed_merge"):
+        assert getattr(lib, name)(ctypes.byref(d), z, z, z, z, z, 0, z, 0.1, z, z, 1 << 30,
+                                  None) == pa.PA_ERR_INVALID_ARG
