@@ -57,3 +57,35 @@ def test_kv_bytes_accounting():
     assert workloads.kv_bytes(w, cl) == 30 * 8 * 128 * 2 * 2
     m = workloads.get("mla")
     assert workloads.kv_bytes(m, cl) == 30 * 576 * 2
+
+
+def test_index_list_workload_structure():
+    # a scaled-down copy of the topk recipe: sorted unique draws below ctx - window,
+    # then the window; only blocks holding a selected token are mapped, each once
+    w = workloads.IndexedWorkload("t", 3, 8, 2, 128, "bf16", 16, 700, 60, 16, 5)
+    inp = workloads.make_indexed(w)
+    sel, table, bs = inp["token_index"], inp["block_table"], w.block_size
+    assert sel.shape == (3, 76) and torch.all(inp["n_sel"] == 76)
+    seen = set()
+    for b in range(3):
+        top, win = sel[b, :60], sel[b, 60:]
+        assert torch.all(top[1:] > top[:-1]) and int(top.min()) >= 0 and int(top.max()) < 700 - 16
+        assert win.tolist() == list(range(700 - 16, 700))
+        need = set((sel[b] // bs).tolist())
+        mapped = {j for j in range(table.shape[1]) if int(table[b, j]) >= 0}
+        assert mapped == need
+        ids = [int(table[b, j]) for j in mapped]
+        assert not (set(ids) & seen) and len(set(ids)) == len(ids)
+        seen |= set(ids)
+    assert seen == set(range(inp["k_cache"].shape[0]))
+
+
+def test_float8_workload_codes_are_finite_e4m3():
+    w = workloads.get("gqa_fp8", batch=2)
+    inp = workloads.make(w)
+    for name in ("k_cache", "v_cache"):
+        codes = inp[name]
+        assert codes.dtype == torch.uint8
+        assert not torch.any((codes & 0x7F) == 0x7F)          # no NaN code
+        vals = codes.view(torch.float8_e4m3fn).float() * inp["k_scale"]
+        assert abs(vals.mean().item()) < 0.05 and 0.8 < vals.std().item() < 1.2
