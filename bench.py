@@ -262,10 +262,10 @@ def cpu_baseline(w, inp, target_s):
     cl = live_lens(w, inp)
     H = w.num_heads if w.kind == "mla" else w.num_q_heads
 
-    def run(nseq, nheads):
+    def run(nseq, nheads, threads=nthreads):
         pairs = np.array([(b, h) for b in range(nseq) for h in range(nheads)], np.int32)
         t0 = time.perf_counter()
-        oracle_rows(w, inp, pairs, nthreads)
+        oracle_rows(w, inp, pairs, threads)
         return time.perf_counter() - t0
 
     # calibrate on the first sequence (all heads), then grow to ~target_s; when the
@@ -283,10 +283,14 @@ def cpu_baseline(w, inp, target_s):
         reps += 1
     sample_cl = cl[:nseq]
     nbytes = workloads.kv_bytes(w, sample_cl) * reps
+    # the same oracle on one thread, over the first sequence (all heads)
+    t_one = max(run(1, H, threads=1), 1e-6)
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "sample": f"first {nseq} of {w.batch} sequences ({int(sample_cl.sum())} tokens, all "
                       f"{H} heads) x {reps} pass(es), float64 C oracle, {dt:.1f} s",
-            "seconds": dt}
+            "value_1thread": workloads.kv_bytes(w, cl[:1]) / t_one / 1e9,
+            "sample_1thread": f"first sequence ({int(cl[0])} tokens, all {H} heads), 1 thread",
+            "seconds": dt + t_one}
 
 
 # ------------------------------------------------------------------ our implementation

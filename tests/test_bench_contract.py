@@ -50,3 +50,15 @@ def test_reference_arm_under_two_ranks():
     lines = json_lines(r.stdout)
     assert len(lines) == 1                   # rank 0 alone prints
     check_line(lines[0], 2)
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    import workloads
+    w = workloads.get("tiny")
+    cb = bench.cpu_baseline(w, workloads.make(w), 0.2)
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
+    assert cb["value_1thread"] > 0 and "1 thread" in cb["sample_1thread"]
