@@ -154,3 +154,31 @@ def test_float8_entry_point_validation(lib):
     for name in ("pa_decode_indexed_partition", "pa_decode_indexed_merge"):
         assert getattr(lib, name)(ctypes.byref(d), z, z, z, z, z, 0, z, 0.1, z, z, 1 << 30,
                                   None) == pa.PA_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    # the boundary is a C ABI: the header compiles as C (and C++), and a C program
+    # links against the library and calls a host-side entry point
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_pa.c"
+    src.write_text(
+        '#include "pa.h"\n#include <stdio.h>\n'
+        "int main(void) {\n"
+        "  pa_desc d = {4, 32, 8, 128, 16, 64, 300, PA_BF16, 10};\n"
+        "  size_t n = pa_workspace_size(&d);\n"
+        '  printf("%zu %s\\n", n, pa_status_string(PA_ERR_UNSUPPORTED));\n'
+        "  return n > 0 ? 0 : 1;\n}\n")
+    libdir = os.path.join(ROOT, "paged_split_kv_attention_b200")
+    exe = tmp_path / "use_pa"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lpa_b200", "-Wl,-rpath," + libdir, "-o", str(exe)],
+                   check=True, capture_output=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "unsupported" in r.stdout
+    subprocess.run(["g++", "-std=c++17", "-fsyntax-only", "-Wall", "-Werror", "-x", "c++",
+                    os.path.join(ROOT, "include", "pa.h")], check=True, capture_output=True)
