@@ -255,6 +255,28 @@ def oracle_rows(w, inp, pairs, nthreads):
                              inp["dtype"], w.v_dim, pairs=pairs, nthreads=nthreads)
 
 
+def parity_sample(w, inp, out_host, n=32, seed=0):
+    """Error of sampled output rows (the longest and shortest sequence plus random
+    ones) against the float64 oracle, with the elementwise tolerance of the tests."""
+    import numpy as np
+    cl = live_lens(w, inp)
+    H = w.num_heads if w.kind == "mla" else w.num_q_heads
+    g = torch.Generator().manual_seed(seed)
+    bs = [int(cl.argmax()), int(cl.argmin())] + torch.randint(0, w.batch, (n - 2,),
+                                                              generator=g).tolist()
+    hs = torch.randint(0, H, (n,), generator=g).tolist()
+    pairs = np.array(list(zip(bs, hs)), np.int32)
+    ref = np.asarray(oracle_rows(w, inp, pairs, os.cpu_count() or 1), np.float64)
+    got = out_host[torch.from_numpy(pairs[:, 0]).long(),
+                   torch.from_numpy(pairs[:, 1]).long()].double().numpy()
+    err = np.abs(got - ref)
+    big = np.abs(ref) >= 0.05
+    return {"rows": n, "max_abs": float(err.max()),
+            "max_rel": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+            "within_tolerance": bool(np.all(err <= 2e-3 + 1e-2 * np.abs(ref))),
+            "tolerance": "|out - oracle| <= 2e-3 + 1e-2 |oracle| elementwise (float64 oracle)"}
+
+
 def cpu_baseline(w, inp, target_s):
     """Time the float64 oracle on a bounded sample (leading sequences of the batch)."""
     import numpy as np
@@ -496,6 +518,12 @@ def run_ours(args, rank, world, local):
         "gpu_launches_note": ("per step: the partition kernel, which also merges" if fused else
                               "per step: the partition kernel + the LSE merge kernel"),
     }
+    if rank == 0 and world == 1:
+        # the last step's output against the oracle on sampled rows (after all timing)
+        try:
+            result["parity"] = parity_sample(w, inp, out.float().cpu())
+        except Exception as e:  # reported, never fatal to the measurement line
+            result["parity"] = {"error": repr(e)[:200]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(w, inp, args.cpu_seconds)
         cb.pop("seconds", None)

@@ -62,3 +62,27 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     cb = bench.cpu_baseline(w, workloads.make(w), 0.2)
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
     assert cb["value_1thread"] > 0 and "1 thread" in cb["sample_1thread"]
+
+
+def test_parity_sample_against_the_oracle():
+    import importlib.util
+    import numpy as np
+    import torch
+    spec = importlib.util.spec_from_file_location("bench_mod2", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    import oracle
+    import workloads
+    w = workloads.get("gqa", batch=3)
+    inp = workloads.make(w)
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    full = oracle.decode(u16(inp["q"]), u16(inp["k_cache"]), u16(inp["v_cache"]),
+                         inp["block_table"].numpy(), inp["context_lens"].numpy(), inp["scale"],
+                         inp["dtype"])
+    exact = torch.from_numpy(np.asarray(full)).to(torch.bfloat16)   # the oracle, rounded
+    r = bench.parity_sample(w, inp, exact.float(), n=12)
+    assert r["within_tolerance"] and r["max_abs"] <= 2e-2 and r["rows"] == 12
+    bad = exact.float().clone()
+    bad[:, :, 5] += 0.5                                              # a wrong dim everywhere
+    r = bench.parity_sample(w, inp, bad, n=12)
+    assert not r["within_tolerance"] and r["max_abs"] >= 0.49
