@@ -1,7 +1,13 @@
 """Benchmark of the paged split-KV decode step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa|long|mixed|mla|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload mixed|long|gqa|mla|tiny|gqa_fp8|topk] [--batch B]
                     [--impl ours|reference]
+
+The default workload is the mixed continuous-batching decode (256 sequences,
+lengths log-uniform in [1, 32768]), the largest single-GPU configuration; the
+long-context one is `--workload long`.  --batch replaces the workload's batch
+size (for profiling a smaller case of the same shapes and length mix).
 
 One step = one paged decode call (partition pass + LSE merge pass) over the
 workload's whole batch, inputs resident in HBM.  The L2 is flushed between
@@ -62,8 +68,10 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="gqa",
+    ap.add_argument("--workload", default="mixed",
                     choices=sorted(list(workloads.WORKLOADS) + list(workloads.INDEXED)))
+    ap.add_argument("--batch", type=int, default=None,
+                    help="replace the workload's batch size (same shapes and length mix)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -112,10 +120,30 @@ def sum_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def get_workload(name, seed_offset=0):
+def get_workload(name, seed_offset=0, batch=None):
     import dataclasses
     w = workloads.INDEXED[name] if name in workloads.INDEXED else workloads.get(name)
+    if batch is not None and batch != w.batch:
+        if getattr(w, "ctx", "").startswith("fixed:"):
+            raise SystemExit(f"--batch: workload {name} has fixed context lengths")
+        w = dataclasses.replace(w, batch=batch)
     return dataclasses.replace(w, seed=w.seed + seed_offset) if seed_offset else w
+
+
+def describe(name, batch=None):
+    """The workload's description, with the batch size replaced when overridden."""
+    d = DESCRIPTIONS[name]
+    return re.sub(r"\bB\d+", f"B{batch}", d, count=1) if batch is not None else d
+
+
+def workload_config(args, w, inp, world):
+    """The `config` object of the JSON line: the workload and how it is timed.
+    Both arms print the same keys and values for the same workload."""
+    return {"workload": describe(args.workload, args.batch), "batch": w.batch,
+            "kv_bytes_per_step_per_gpu": workloads.kv_bytes(w, live_lens(w, inp)),
+            "tokens_per_step_per_gpu": int(live_lens(w, inp).sum()),
+            "parallelism": f"replicas x{world} (independent batches)",
+            "l2": "flushed between steps (512 MiB write + 512 MiB read of another buffer)"}
 
 
 def make_inputs(w):
@@ -127,10 +155,10 @@ def live_lens(w, inp):
     return inp["n_sel"] if w.kind == "gqa_indexed" else inp["context_lens"]
 
 
-def rank_workload(name, rank, world):
+def rank_workload(name, rank, world, batch=None):
     """The workload a rank decodes: the same shapes on every rank, its own seeded
     batch of independent sequences when several ranks run (weak scaling)."""
-    return get_workload(name, 7919 * rank if world > 1 else 0)
+    return get_workload(name, 7919 * rank if world > 1 else 0, batch)
 
 
 def barrier(world):
@@ -321,7 +349,7 @@ def run_ours(args, rank, world, local):
     import paged_split_kv_attention_b200 as pa
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = rank_workload(args.workload, rank, world)
+    w = rank_workload(args.workload, rank, world, args.batch)
     inp = make_inputs(w)
     kv_bytes = workloads.kv_bytes(w, live_lens(w, inp))
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
@@ -505,14 +533,10 @@ def run_ours(args, rank, world, local):
         "us_per_step": round(ms_per_step * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": inp["dtype"], "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool)",
-        "config": {"workload": DESCRIPTIONS[args.workload], "batch": w.batch,
-                   "kv_bytes_per_step_per_gpu": kv_bytes,
-                   "tokens_per_step_per_gpu": int(live_lens(w, inp).sum()),
-                   "partitions": parts,
+        "config": workload_config(args, w, inp, world),
+        "launch": {"partitions": parts,
                    "merge": ("single-pass (pa_decode_fused: one launch)" if fused else
-                             "separate kernel (programmatic dependent launch)"),
-                   "parallelism": f"replicas x{world} (independent batches)",
-                   "l2": "flushed between steps (512 MiB write + 512 MiB read of another buffer)"},
+                             "separate kernel (programmatic dependent launch)")},
         "roofline": roofline, "clocks": clocks, "e2e": e2e,
         "gpu_launches": (1 if fused else 2) * K,
         "gpu_launches_note": ("per step: the partition kernel, which also merges" if fused else
@@ -545,7 +569,7 @@ def run_reference(args, rank, world):
         return
     import numpy as np
 
-    w = get_workload(args.workload)
+    w = get_workload(args.workload, batch=args.batch)
     inp = make_inputs(w)
     nthreads = os.cpu_count() or 1
     cl = live_lens(w, inp)
@@ -579,11 +603,10 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / len(times) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool)",
-        "config": {"workload": DESCRIPTIONS[args.workload], "batch": w.batch,
-                   "sample_sequences": nseq},
+        "config": workload_config(args, w, inp, world),
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": nthreads,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, "sample_sequences": nseq},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

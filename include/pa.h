@@ -149,8 +149,9 @@ pa_status pa_decode_merge(const pa_desc *desc, const void *q, const void *k_cach
  * CUDA graph may be replayed.  The result equals pa_decode's up to the order of
  * the merge's fp32 sums (the pieces are the same), and repeated calls on the
  * same inputs are bitwise identical.  Two calls in flight at once must not share
- * a workspace.  Errors as pa_decode; a call that reported PA_ERR_TIMEOUT may
- * leave counters of its own epoch behind, which no later call reads. */
+ * a workspace.  Errors as pa_decode.  A piece whose wait timed out
+ * (PA_ERR_TIMEOUT) still counts itself in, so every counter returns to zero
+ * even then and a captured graph may be replayed after the error is cleared. */
 pa_status pa_decode_fused(const pa_desc *desc, const void *q, const void *k_cache,
                           const void *v_cache, const int32_t *block_table,
                           const int32_t *context_lens, float scale, void *out, void *workspace,
@@ -248,13 +249,16 @@ int pa_default_partitions(int kind, int head_dim);
  * current device since the last reset (PA_OK if none); reset != 0 clears it. */
 pa_status pa_device_status(void *stream, int reset);
 
-/* Test hook for the kernels' timeout path (not for production use).  While
- * enabled (process-wide, for GQA calls launched afterwards), one warp of the GQA
- * partition pass waits on an mbarrier that nothing completes before it issues
- * any copy; its bounded wait gives up after about one second, records
- * PA_ERR_TIMEOUT (readable through pa_device_status) and the warp leaves, so the
- * call's output is incomplete but the CUDA context stays usable.  enable = 0
- * restores normal operation. */
+/* Test hook for the kernels' timeout path (not for production use).  Sets a
+ * flag in device memory of the current device (a synchronous copy: call it
+ * between launches).  While it is set, one warp of every partition pass that
+ * runs (GQA: warp 0 of CTA 0; MLA: the copy-issuing warp of CTA 0) waits on an
+ * mbarrier that nothing completes before it issues any copy; its bounded wait
+ * gives up after about one second, records PA_ERR_TIMEOUT (readable through
+ * pa_device_status) and the CTA finishes without it, so the call's output is
+ * incomplete but the CUDA context stays usable.  The kernels read the flag when
+ * they run, so a launch captured in a CUDA graph follows the flag's value at
+ * replay time.  enable = 0 restores normal operation. */
 void pa_test_inject_stall(int enable);
 
 /* pa_decode without a workspace argument, for callers that cannot allocate
@@ -271,7 +275,10 @@ void pa_test_inject_stall(int enable);
  *
  *   - The first call on each device looks up the buffer's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.  Later calls reuse the address.
+ *     before any stream capture.  Later calls reuse the address.  The address
+ *     belongs to the CUDA context it was looked up in: after a device reset
+ *     (cudaDeviceReset) or under another context, the next call looks it up
+ *     again, and that call too should come before any stream capture.
  *   - A call whose workspace (pa_workspace_size) exceeds the buffer returns
  *     PA_ERR_TOO_LARGE before launching anything.
  *   - All calls on a device share the one buffer, and it keeps the last call's

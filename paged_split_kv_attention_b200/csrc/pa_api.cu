@@ -334,10 +334,6 @@ cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int seg
 int min_tiles_gqa(int G) { return G > 2 ? G : 2; }
 constexpr int kMinTilesMla = 16;
 
-// Test hook (pa_test_inject_stall): makes the next GQA partition launches take
-// their timeout path.
-std::atomic<int> g_stall_test{0};
-
 // kFused: the partition kernel also merges (the last piece of each split segment),
 // so no merge grid is launched
 enum Pass { kPartition = 1, kMerge = 2, kBoth = 3, kFused = 4 };
@@ -413,7 +409,6 @@ pa_status run_gqa(int passes, const pa_desc *d, const void *q, const void *k, co
     p.max_sel = max_sel;
     p.k_cache = k;
     p.v_cache = v;
-    p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     p.min_tiles = d->num_partitions == 0 ? min_tiles_gqa(pl.G) : 0;
     p.seg_ctr = reinterpret_cast<unsigned long long *>(w + pl.off_ctr);
     p.seg_units = mode == kModeIndexed ? 0 : kSegUnits;
@@ -708,7 +703,10 @@ int pa_default_partitions(int kind, int head_dim) {
   return default_mla_parts();
 }
 
-void pa_test_inject_stall(int enable) { g_stall_test.store(enable ? 1 : 0); }
+void pa_test_inject_stall(int enable) {
+  const int v = enable ? 1 : 0;
+  (void)cudaMemcpyToSymbol(pa::g_stall_test, &v, sizeof(int));
+}
 
 pa_status pa_device_status(void *stream, int reset) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
@@ -742,27 +740,67 @@ const char *pa_status_string(pa_status s) {
 // Scratch of pa_decode_static: a fixed device buffer in the library itself, for
 // callers that cannot allocate device memory.  Host code must not pass the
 // symbol itself to a kernel (on the host it names a shadow variable, not device
-// memory); its device address is looked up once per device below.
+// memory); its device address is looked up below, once per CUDA context (one per
+// device unless the device is reset).
 static __device__ __align__(256) unsigned char g_pa_static_scratch[PA_STATIC_SCRATCH_BYTES];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mu;
-void *g_static_ptr[kMaxDevices] = {};
+// The address is valid in the CUDA context it was looked up in.  A device reset
+// destroys that context (and a driver-API caller may make another one current),
+// so the cache is keyed by the unique id of the current context (cuCtxGetId),
+// never by the device ordinal: a context created after a reset gets a new id and
+// a fresh lookup.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
 
-// Device address of the static scratch on the current device (looked up on the
-// first call per device), or nullptr on error.
+template <typename F>
+F driver_fn(const char *name) {
+  void *ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &ptr, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(ptr);
+}
+
+// Unique id of the calling thread's current context, or 0 if there is none.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+constexpr int kMaxContexts = 64;
+std::mutex g_static_mu;
+unsigned long long g_static_ctx[kMaxContexts] = {};
+void *g_static_ptr[kMaxContexts] = {};
+int g_static_n = 0;
+
+// Device address of the static scratch in the current context (looked up on the
+// first call in each context), or nullptr on error.
 void *static_scratch_address() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_pa_static_scratch) != cudaSuccess || !ptr) return nullptr;
-    g_static_ptr[dev] = ptr;
+  unsigned long long id = current_context_id();
+  for (int i = 0; id != 0 && i < g_static_n; ++i)
+    if (g_static_ctx[i] == id) return g_static_ptr[i];
+  // with no context current yet, the lookup makes the device's primary one current
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_pa_static_scratch) != cudaSuccess || !ptr) return nullptr;
+  if (id == 0) id = current_context_id();
+  if (id != 0 && g_static_n < kMaxContexts) {
+    g_static_ctx[g_static_n] = id;
+    g_static_ptr[g_static_n] = ptr;
+    ++g_static_n;
   }
-  return g_static_ptr[dev];
+  return ptr;
 }
 
 }  // namespace

@@ -22,6 +22,16 @@ namespace pa {
 // Device status word: first error recorded by any kernel (0 = none).
 __device__ int g_status;
 
+// Test hook of the timeout path (pa_test_inject_stall): while nonzero, one warp
+// of every partition launch waits on a barrier that nothing completes before it
+// issues any copy.  Read by the kernels when they run, so a launch captured in a
+// CUDA graph sees the value current at replay time.
+__device__ int g_stall_test;
+
+__device__ __forceinline__ bool stall_test_enabled() {
+  return *reinterpret_cast<volatile int *>(&g_stall_test) != 0;
+}
+
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_status, 0, code); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -87,8 +87,7 @@ struct GqaParams {
   int tiles_per_block;          // bs / 16
   int parts;                    // gridDim.x
   float scale_log2;             // scale * log2(e)
-  int stall_test;               // test hook: warp 0 of CTA 0 waits on a barrier nothing completes
-  int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
+  int min_tiles;               // > 0: at least this many tiles per piece (automatic launches)
   float v_scale;                // value scale of a float8 KV cache (1 otherwise)
   // index-list decode (MODE 2): context_lens holds the selected counts n_sel
   const int32_t *token_index;   // [B][max_sel] token positions
@@ -306,12 +305,15 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   __syncthreads();
   if (wb >= we) return;
 
-  if (p.stall_test && c == 0 && warp == 0) {
+  bool aborted = false;
+  if (c == 0 && warp == 0 && stall_test_enabled()) {
     // Test hook for the timeout path: wait on this warp's first stage barrier
     // before anything is issued into it, so that nothing can complete the wait.
     // The bounded wait gives up, records PA_ERR_TIMEOUT and raises the CTA's
-    // abort flag; with no copy in flight the warp simply leaves.
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[0], 0, abort_flag))) return;
+    // abort flag.  The warp then runs its piece as aborted: it issues and waits
+    // for nothing, and in the single-pass form it still counts itself in at its
+    // split segments so that their counters return to zero.
+    aborted = !__all_sync(0xffffffffu, mbar_wait(&full[0], 0, abort_flag));
   }
 
   const uint64_t policy = l2_evict_first_policy();
@@ -407,7 +409,8 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     ++issued;
   };
-  for (int s = 0; s < R; ++s) issue_next();
+  if (!aborted)
+    for (int s = 0; s < R; ++s) issue_next();
 
   const int g = lane >> 2;          // fragment row group
   const int tq = lane & 3;          // thread in quad
@@ -424,7 +427,6 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
   (void)tm_k;
   (void)tm_v;
   int ctx = clamp_ctx(__ldg(&p.context_lens[b]), cap);
-  bool aborted = false;
 
   long long split_seg[2] = {0, 0}, split_first[2] = {0, 0};
   int split_tiles[2] = {0, 0}, n_split = 0;
@@ -708,7 +710,12 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       }
   }
 
-  if (FUSED && n_split > 0 && !aborted) {
+  // An aborted piece (a wait timed out) still counts itself in, so that every
+  // counter it shares returns to zero and a replayed graph, which reuses the
+  // epoch, starts from a clean count; the segment is then merged only if the
+  // last arrival is a piece that completed (the output is invalid either way and
+  // the status word says so).
+  if (FUSED && n_split > 0) {
     __threadfence();                     // every lane's partial rows before the arrivals
     __syncwarp();
 #pragma unroll
@@ -718,7 +725,7 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
       const int g0 = piece_of(split_first[i], TP, pieces);
       const int g1 = piece_of(split_first[i] + split_tiles[i] - 1, TP, pieces);
       const int expected = pieces_with_tiles(g0, g1, TP, pieces, lane);
-      if (segment_arrive_last(p.seg_ctr + sg, p.epoch, expected, lane)) {
+      if (segment_arrive_last(p.seg_ctr + sg, p.epoch, expected, lane) && !aborted) {
         const long long sb = sg / p.Hkv, skv = sg - sb * p.Hkv;
         uint16_t *rows = reinterpret_cast<uint16_t *>(p.out) + (sb * p.Hq + skv * p.G) * D;
         merge_segment_warp<D, 8 * NT, BF16>(p.part_o, p.part_lse, sg, p.G, g0, g1, TP, pieces,

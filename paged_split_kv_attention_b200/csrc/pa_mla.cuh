@@ -159,7 +159,8 @@ enum MlaBar {
   kQFull = 10,      // query of sequence k in TMEM + shared memory (4 warps)
   kQEmpty = 11,     // last score MMA of sequence k done (commit)
   kOFree = 12,      // epilogue has read O (4 warps)
-  kFinal = 13       // all MMAs of this CTA done (commit)
+  kFinal = 13,      // all MMAs of this CTA done (commit)
+  kStall = 14       // test hook only: nothing ever arrives here
 };
 
 __global__ void __launch_bounds__(kMlaThreads, 1)
@@ -261,6 +262,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p)
     cur.init(p, b_first, j_first, ntiles);
     int issued = 0;
     bool aborted = false;
+    if (blockIdx.x == 0 && stall_test_enabled()) {
+      // Test hook for the timeout path: wait, before anything is issued, on a
+      // barrier that nothing completes.  The bounded wait gives up after about a
+      // second, records PA_ERR_TIMEOUT and raises the CTA's abort flag, which
+      // ends the issuer's and the softmax warps' waits too; no copy or MMA is in
+      // flight, and tensor memory is released as usual.
+      const bool got = lane != 0 || mbar_wait_idle(&bar[kStall], 0, abort_flag);
+      aborted = !__all_sync(0xffffffffu, got);
+    }
     if (lane == 0) prefetch_tensormap(&tm_lat);
     for (int base = 0; base < ntiles && !aborted; base += 32) {
       const int n = min(32, ntiles - base);
