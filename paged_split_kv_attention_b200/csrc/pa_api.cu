@@ -84,6 +84,23 @@ bool make_map_3d_halves(CUtensorMap *m, const void *base, bool bf16, uint64_t ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// MLA latent pool (or query) [rows][576] bf16 viewed as (64 dims, rows, 9 slabs): the slabs
+// are 128 bytes apart in a row.  A box of 64 x box_rows x box_slabs lands as
+// [box_slabs][box_rows][64] with 128 B swizzle: whole slabs of a token range, in
+// the layout that 2-D boxes of one 64-dim slab give one slab at a time.
+bool make_map_latent_slabs(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows,
+                           uint32_t box_slabs) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, pa::kMlaDk / 64};
+  cuuint64_t strides[2] = {pa::kMlaDk * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_slabs};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Float8 KV cache: one byte per element, rows of `inner` bytes.
 bool make_map_2d_u8(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows,
                     uint32_t box_inner, uint32_t box_rows) {
@@ -327,12 +344,12 @@ cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int seg
 // does not cut a short tile stream into pieces much smaller than the partial
 // output each piece writes: a piece leaves G x D fp32 (GQA: one 16-token K+V tile
 // is 16 x D x 4 bytes, so G tiles per piece keep partials at or below the KV
-// bytes read; at least 2) or 128 x 512 fp32 (MLA: 16 tiles of 64 tokens).  A
+// bytes read; at least 2) or 128 x 512 fp32 (MLA: 8 tiles of 128 tokens).  A
 // single short sequence or a single kv head would otherwise spend more on
 // partials and their merge than on the KV.  An explicit partition count is used
 // as given.
 int min_tiles_gqa(int G) { return G > 2 ? G : 2; }
-constexpr int kMinTilesMla = 16;
+constexpr int kMinTilesMla = 8;   // tiles of 128 tokens
 
 // kFused: the partition kernel also merges (the last piece of each split segment),
 // so no merge grid is launched
@@ -447,19 +464,39 @@ struct MlaPlan {
   size_t off_lse = 0, off_o = 0, bytes = 0;
 };
 
-// Pieces whose two CTAs can all be resident at once (one CTA per SM).
+// Launch configuration of the MLA partition pass: clusters of two CTAs (one CTA
+// pair per piece), one CTA per SM by its shared memory.
+cudaLaunchConfig_t mla_launch_config(int parts, cudaStream_t st, cudaLaunchAttribute *attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * parts), 1, 1);
+  cfg.blockDim = dim3(pa::kMlaThreads, 1, 1);
+  cfg.dynamicSmemBytes = pa::MlaLayout::bytes();
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Pieces (CTA pairs) that can all be resident at once: a pair must fit on two
+// SMs of one GPU processing cluster, so this can be fewer than SMs / 2.
 int default_mla_parts() {
   const size_t smem = pa::MlaLayout::bytes();
   if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return -1;
-  const int sms = sm_count();
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pa::mla_decode_kernel,
-                                                    pa::kMlaThreads, smem) != cudaSuccess ||
-      per_sm <= 0)
-    per_sm = 1;
-  return sms * per_sm / 2 > 0 ? sms * per_sm / 2 : -1;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = mla_launch_config(1, nullptr, attr);
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, pa::mla_decode_kernel, &cfg) != cudaSuccess ||
+      clusters <= 0) {
+    const int sms = sm_count();
+    return sms >= 2 ? sms / 2 : -1;
+  }
+  return clusters;
 }
 
 pa_status plan_mla(const pa_mla_desc *d, MlaPlan *pl) {
@@ -508,9 +545,22 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
   uint8_t *w = static_cast<uint8_t *>(ws);
 
   if (passes & kPartition) {
-    CUtensorMap tl;
-    if (!make_map_2d(&tl, lat, true, pa::kMlaDk, uint64_t(d->num_blocks) * d->block_size, 64,
-                     pa::kMlaBox))
+    // block sizes that are multiples of 64: whole-slab boxes of a CTA's 64 tokens
+    // (the stage's 9 slabs in one copy, the value slabs in two); else 32-row
+    // boxes of one 64-dim slab each
+    const bool wide = d->block_size % 64 == 0;
+    CUtensorMap ta, tb;
+    const uint64_t rows = uint64_t(d->num_blocks) * d->block_size;
+    if (wide ? !(make_map_latent_slabs(&ta, lat, rows, 64, pa::MlaLayout::kSlabs) &&
+                 make_map_latent_slabs(&tb, lat, rows, 64, 2))
+             : !make_map_2d(&ta, lat, true, pa::kMlaDk, rows, 64, pa::kMlaBox))
+      return PA_ERR_CUDA;
+    if (!wide) tb = ta;
+    // the query [B * 128 heads][576] in the same slab view: a 64-head x 5-slab box
+    // is the shared-memory part of the score MMA's A operand
+    CUtensorMap tq;
+    if (!make_map_latent_slabs(&tq, q, uint64_t(d->batch) * pa::kMlaHeads, 64,
+                               pa::MlaLayout::kQSlabs))
       return PA_ERR_CUDA;
     pa::MlaParams p;
     p.q = static_cast<const uint16_t *>(q);
@@ -526,16 +576,14 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     p.parts = pl.parts;
     p.min_tiles = d->num_partitions == 0 ? kMinTilesMla : 0;
     p.scale_log2 = scale * kLog2e;
+    p.wide = wide ? 1 : 0;
     const size_t smem = pa::MlaLayout::bytes();
     if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return PA_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pl.parts), 1, 1);
-    cfg.blockDim = dim3(pa::kMlaThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, tl, p) != cudaSuccess)
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = mla_launch_config(pl.parts, st, attr);
+    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, ta, tb, tq, p) != cudaSuccess)
       return PA_ERR_CUDA;
   }
   if (passes & kMerge) {
