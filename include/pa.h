@@ -95,7 +95,7 @@ typedef struct {
 } pa_desc;
 
 /* Shape of an MLA absorbed decode call.  Supported: num_heads 128, kv_dim 576,
- * v_dim 512, block_size a multiple of 32 up to 1024, dtype PA_BF16,
+ * v_dim 512, block_size a multiple of 16 up to 1024, dtype PA_BF16,
  * 0 <= batch <= 32768.
  * num_partitions counts CTA pairs (0 = as many as can be resident). */
 typedef struct {

@@ -349,7 +349,7 @@ cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int seg
 // partials and their merge than on the KV.  An explicit partition count is used
 // as given.
 int min_tiles_gqa(int G) { return G > 2 ? G : 2; }
-constexpr int kMinTilesMla = 8;   // tiles of 128 tokens
+constexpr int kMinTilesMla = 11;  // tiles of 96 tokens
 
 // kFused: the partition kernel also merges (the last piece of each split segment),
 // so no merge grid is launched
@@ -545,18 +545,17 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
   uint8_t *w = static_cast<uint8_t *>(ws);
 
   if (passes & kPartition) {
-    // block sizes that are multiples of 64: whole-slab boxes of a CTA's 64 tokens
-    // (the stage's 9 slabs in one copy, the value slabs in two); else 32-row
-    // boxes of one 64-dim slab each
-    const bool wide = d->block_size % 64 == 0;
-    CUtensorMap ta, tb;
+    // A CTA's 48 tokens of a tile: one 3-D box of whole slabs when they lie in one
+    // block, else 2-D boxes of 16 or 32 rows of one 64-dim slab each (block sizes
+    // are multiples of 16, so no 16-row group crosses a block)
+    CUtensorMap ta, ta32, tw9, tw2;
     const uint64_t rows = uint64_t(d->num_blocks) * d->block_size;
-    if (wide ? !(make_map_latent_slabs(&ta, lat, rows, 64, pa::MlaLayout::kSlabs) &&
-                 make_map_latent_slabs(&tb, lat, rows, 64, 2))
-             : !make_map_2d(&ta, lat, true, pa::kMlaDk, rows, 64, pa::kMlaBox))
+    if (!make_map_2d(&ta, lat, true, pa::kMlaDk, rows, 64, pa::kMlaBox) ||
+        !make_map_2d(&ta32, lat, true, pa::kMlaDk, rows, 64, 2 * pa::kMlaBox) ||
+        !make_map_latent_slabs(&tw9, lat, rows, pa::kMlaHalf, pa::MlaLayout::kSlabs) ||
+        !make_map_latent_slabs(&tw2, lat, rows, pa::kMlaHalf, 2))
       return PA_ERR_CUDA;
-    if (!wide) tb = ta;
-    // the query [B * 128 heads][576] in the same slab view: a 64-head x 5-slab box
+    // the query [B * 128 heads][576] in the same slab view: a 64-head x 4-slab box
     // is the shared-memory part of the score MMA's A operand
     CUtensorMap tq;
     if (!make_map_latent_slabs(&tq, q, uint64_t(d->batch) * pa::kMlaHeads, 64,
@@ -564,6 +563,7 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
       return PA_ERR_CUDA;
     pa::MlaParams p;
     p.q = static_cast<const uint16_t *>(q);
+    p.lat = static_cast<const uint16_t *>(lat);
     p.block_table = bt;
     p.context_lens = cl;
     p.out = out;
@@ -576,14 +576,13 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     p.parts = pl.parts;
     p.min_tiles = d->num_partitions == 0 ? kMinTilesMla : 0;
     p.scale_log2 = scale * kLog2e;
-    p.wide = wide ? 1 : 0;
     const size_t smem = pa::MlaLayout::bytes();
     if (cudaFuncSetAttribute(pa::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return PA_ERR_CUDA;
     cudaLaunchAttribute attr[1];
     const cudaLaunchConfig_t cfg = mla_launch_config(pl.parts, st, attr);
-    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, ta, tb, tq, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, pa::mla_decode_kernel, ta, ta32, tw9, tw2, tq, p) != cudaSuccess)
       return PA_ERR_CUDA;
   }
   if (passes & kMerge) {

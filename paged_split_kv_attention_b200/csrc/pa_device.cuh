@@ -148,6 +148,14 @@ __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *m
 }
 
 // Prefetch a 2-D tile of a tensor map into L2 (no shared memory, no completion).
+// Prefetch `bytes` (a multiple of 16) from a 16-byte aligned global address into
+// L2 with a cache policy (no shared memory, no completion).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes, uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(p), "r"(bytes),
+               "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),

@@ -20,38 +20,44 @@
 // the result rows.
 //   - Heads: CTA r owns heads [64r, 64r+64) (the A rows: the query for the score
 //     MMA, P for the value MMA).
-//   - Scores: S = Q C^T, M = 128 heads, N = 128 tokens, K = 576.  CTA r stages
-//     its own 64 tokens of the tile (all 576 dims, 72 KB) as its half of B.  The
-//     scores are computed once for the pair, at N = 128.
+//   - Scores: S = Q C^T, M = 128 heads, N = 96 tokens, K = 576.  CTA r stages
+//     its own 48 tokens of the tile (all 576 dims, 54 KB) as its half of B.  The
+//     scores are computed once for the pair.  (A 2-SM MMA of M = 128 takes the
+//     same time for every N up to 192, measured on B200, so 96 tokens cost as
+//     much per instruction as 128; the smaller tile buys a third stage.)
 //   - Values: O += P V, M = 128 heads, N = 256 dims per MMA, two MMAs for the
-//     512 dims, K = the tile's 128 tokens.  Each CTA supplies 128 of every 256
-//     dims (B is split by N), for all 128 tokens: its own tokens are staged
+//     512 dims, K = the tile's 96 tokens.  Each CTA supplies 128 of every 256
+//     dims (B is split by N), for all 96 tokens: its own tokens are staged
 //     already, and the other CTA's tokens are fetched for the CTA's value dims
-//     only (32 KB, an L2 hit: the other CTA has just loaded them from HBM)
-//     into the slabs of the stage that only the score MMA needed.
+//     only (24 KB, an L2 hit: the other CTA has just loaded them from HBM) into
+//     the slabs of the stage that only the score MMA needed.
 // So the latent is read from HBM once, the scores are not recomputed, and each
-// SM stages 72 KB per 128 tokens.
+// SM stages 54 KB per 96 tokens.  Three stages let the copies of two tiles run
+// while the third is scored and mixed.
 //
 // Tensor memory per CTA (512 columns, "2x2" layout of a 2-SM M=128 result: lane
 // l < 64 holds head l with the first half of the columns, lane 64 + l the same
 // head with the second half):
-//   [0, 128)    two score buffers of 64 columns (64 heads x 128 tokens)
-//   [128, 256)  query dims [0, 256) as the A operand of the score MMA (each head's
-//               row present in lanes l and 64 + l)
+//   [0, 96)     two score buffers of 48 columns (64 heads x 96 tokens), tile n in
+//               buffer n % 2, each released as soon as the softmax warps have
+//               read it, so a tile's scores are taken while the previous tile's
+//               softmax runs
+//   [96, 256)   query dims [0, 320) as the A operand of the score MMA (each
+//               head's row present in lanes l and 64 + l)
 //   [256, 512)  value accumulator: 64 heads x 512 dims
-// Shared memory per CTA: two 72 KB latent stages, query dims [256, 576) (40 KB),
-// P as a bf16 hi + lo pair (2 x 16 KB, the A operand of the value MMA).
+// Shared memory per CTA: three 54 KB latent stages, query dims [320, 576)
+// (32 KB), and P as a bf16 hi + lo pair (24 KB, the A operand of the value MMA).
 //
-// Warp roles (192 threads per CTA).  Warps 0-3 (thread t: head 64r + t % 64,
-// token half t / 64 of each tile): query loads, the online softmax in log2 units
-// (each head's two threads agree on the running max through shared memory, with
-// a lazily raised max), P as bf16 hi + lo (about 16 significant bits: a single
-// bf16 copy biases the value mix by up to 2^-9 per weight), zeroing value rows
-// past a ragged end, and the epilogue.  Warp 4 issues the TMA loads: its own
-// tokens (completion counted on the rank-0 CTA's barrier, so that the MMA issuer
-// sees both halves land), and, once the tile's scores are done, the other CTA's
-// tokens for its value dims.  Warp 5 of the rank-0 CTA issues every MMA from one
-// thread.  Every wait is bounded.
+// Warp roles (320 threads per CTA).  Warps 0-7 (four threads per head: token
+// half hh and column group cg of each tile, 24 tokens each): query loads, the
+// online softmax in log2 units (a head's four threads agree on the running max
+// through shared memory, with a lazily raised max), P as bf16 hi + lo (about 16
+// significant bits: a single bf16 copy biases the value mix by up to 2^-9 per
+// weight), zeroing value rows past a ragged end, and the epilogue.  Warp 8
+// issues the TMA loads: its own tokens (completion counted on the rank-0 CTA's
+// barrier, so that the MMA issuer sees both halves land), and, once the tile's
+// scores are done, the other CTA's tokens for its value dims.  Warp 9 of the
+// rank-0 CTA issues every MMA from one thread.  Every wait is bounded.
 #pragma once
 
 #include "pa_device.cuh"
@@ -59,18 +65,32 @@
 
 namespace pa {
 
-constexpr int kMlaTile = 128;             // tokens per tile (the pair's)
-constexpr int kMlaHalf = 64;              // tokens of a tile staged by each CTA
-constexpr int kMlaBox = 32;               // rows per TMA box (block sizes: multiples of 32)
+constexpr int kMlaTile = 96;              // tokens per tile (the pair's)
+constexpr int kMlaHalf = 48;              // tokens of a tile staged by each CTA
+constexpr int kMlaBox = 16;               // rows per TMA box (block sizes: multiples of 16)
+constexpr int kMlaBoxes = kMlaHalf / kMlaBox;   // boxes per CTA half tile
 constexpr int kMlaHeads = 128;
 constexpr int kMlaDk = 576;
 constexpr int kMlaDv = 512;
-constexpr int kMlaStages = 2;
-constexpr int kMlaThreads = 192;
+constexpr int kMlaStages = 3;
+#ifndef PA_MLA_LOOKAHEAD
+#define PA_MLA_LOOKAHEAD 2
+#endif
+constexpr int kMlaLookahead = PA_MLA_LOOKAHEAD;   // own-token tiles issued past the next fetch
+#ifndef PA_MLA_PREFETCH
+#define PA_MLA_PREFETCH 2
+#endif
+constexpr int kMlaPrefetch = PA_MLA_PREFETCH;     // tiles ahead whose own rows are pulled into L2
+constexpr int kMlaSoftmaxWarps = 8;       // warps 0-7: softmax and epilogue
+constexpr int kMlaProducer = 8;           // warp 8: copy issue
+constexpr int kMlaIssuer = 9;             // warp 9: MMA issue (rank 0), TMEM allocation
+constexpr int kMlaThreads = 32 * (kMlaSoftmaxWarps + 2);
+constexpr int kMlaTok = kMlaHalf / 2;     // tokens of a tile per softmax thread
 constexpr int kMlaRescale = 8;            // raise the running max only past 2^8 growth
 
 struct MlaParams {
   const uint16_t *q;            // [B][128][576]
+  const uint16_t *lat;          // [nb * bs][576] latent rows (L2 prefetches)
   const int32_t *block_table;   // [B][mbs]
   const int32_t *context_lens;  // [B]
   void *out;                    // [B][128][512] bf16
@@ -80,39 +100,39 @@ struct MlaParams {
   int parts;                    // pieces (CTA pairs)
   int min_tiles;                // > 0: at least this many tiles per piece (automatic launches)
   float scale_log2;
-  int wide;                     // block size a multiple of 64: a CTA's 64 tokens of a tile lie
-                                // in one block and move as whole-slab 3-D boxes
 };
 
 struct MlaLayout {
-  static constexpr int kSlab = kMlaHalf * 128;            // 64 rows x 64 bf16 = 8 KB
+  static constexpr int kSlab = kMlaHalf * 128;            // 48 rows x 64 bf16 = 6 KB
   static constexpr int kSlabs = kMlaDk / 64;              // 9 slabs per staged half tile
-  static constexpr int kStage = kSlabs * kSlab;           // 72 KB
-  static constexpr int kQSlabs = 5;                       // query dims [256, 576)
+  static constexpr int kStage = kSlabs * kSlab;           // 54 KB
+  static constexpr int kHSlab = 64 * 128;                 // 64 head rows x 64 bf16 = 8 KB
+  static constexpr int kQSlabs = 4;                       // query dims [320, 576)
   static constexpr int stage = 0;
   static constexpr int qs = stage + kMlaStages * kStage;
-  // P pool: slabs 0, 1 = P hi of token half 1 for tiles of even / odd index, 2, 3 =
-  // P lo of token halves 0, 1; P hi of token half 0 goes into slab 8 of the tile's
-  // own stage (the rope dims, free once the tile's scores are done)
-  static constexpr int ps = qs + kQSlabs * kSlab;
-  static constexpr int bars = ps + 4 * kSlab;
-  static constexpr int nbars = 17;
-  static constexpr int xch = bars + nbars * 8;            // float xm[2][128], xl[128]
-  static constexpr int misc = xch + 3 * 128 * 4;         // tmem base, abort, scan, start
+  // P pool (64 head rows each, K-major, 128-byte swizzle): slab 0 = P hi of tokens
+  // [0, 64), slab 2 = P lo of tokens [0, 64), slab 1 = P hi of tokens [64, 96) in
+  // its first 64 bytes of every row and P lo of the same tokens in the last 64
+  static constexpr int ps = qs + kQSlabs * kHSlab;
+  static constexpr int bars = ps + 3 * kHSlab;
+  static constexpr int nbars = 23;
+  static constexpr int xch = bars + nbars * 8;            // float xm[2][2][128], xl[2][128]
+  static constexpr int misc = xch + 6 * 128 * 4;         // tmem base, abort, scan, start
   static constexpr int end = misc + 128;
   static constexpr size_t bytes() { return 1024 + end; }
-  static_assert(kStage % 1024 == 0 && qs % 1024 == 0 && ps % 1024 == 0,
+  static_assert(kStage % 1024 == 0 && kSlab % 1024 == 0 && qs % 1024 == 0 && ps % 1024 == 0,
                 "swizzled tiles need 1 KB alignment");
 };
 static_assert(MlaLayout::bytes() <= 232448, "shared memory per CTA");
 
 // Tensor memory columns (exactly 512, allocated for the pair)
-constexpr int kTmS = 0;        // score buffers at 0, 64
-constexpr int kTmQ = 128;      // query dims [0, 256): 16 k-steps x 8 columns
-constexpr int kQTmemDims = 256;
+constexpr int kTmS = 0;        // score buffers at 0 and 48: 48 columns each
+constexpr int kTmQ = 96;       // query dims [0, 320): 20 k-steps x 8 columns
+constexpr int kQTmemDims = 320;
 constexpr int kTmO = 256;      // value accumulator: dims block 0 at 256, block 1 at 384
+static_assert(kTmQ + kQTmemDims / 2 <= kTmO && kTmS + 2 * kMlaHalf <= kTmQ, "tensor memory map");
 
-// tiles of 128 tokens in a sequence of c tokens (c clamped to [0, cap])
+// tiles of 96 tokens in a sequence of c tokens (c clamped to [0, cap])
 __device__ __forceinline__ int mla_tiles(int c, int cap) {
   return (min(max(c, 0), cap) + kMlaTile - 1) / kMlaTile;
 }
@@ -148,8 +168,9 @@ struct MlaCursor {
   }
 };
 
-// Cache row of the 32-token box k (0..3) of tile j of sequence b: -1 for a block
-// id out of range, -2 for a box that lies wholly past the context (not loaded).
+// Cache row of the 16-token box k (0..5: boxes 0-2 are the rank-0 CTA's half, 3-5
+// the other's) of tile j of sequence b: -1 for a block id out of range, -2 for a
+// box that lies wholly past the context (not loaded).
 __device__ __forceinline__ int mla_box_row(const MlaParams &p, int b, int j, int k, int ctx) {
   const int t = j * kMlaTile + k * kMlaBox;
   if (t >= ctx) return -2;
@@ -158,7 +179,7 @@ __device__ __forceinline__ int mla_box_row(const MlaParams &p, int b, int j, int
   return blk * p.bs + t % p.bs;
 }
 
-// Tokens of the tile's half `half` (0: the rank-0 CTA's 64, 1: the other's) that
+// Tokens of the tile's half `half` (0: the rank-0 CTA's 48, 1: the other's) that
 // lie inside a context of ctx tokens.
 __device__ __forceinline__ int mla_half_tokens(int ctx, int j, int half) {
   return min(max(ctx - j * kMlaTile - half * kMlaHalf, 0), kMlaHalf);
@@ -167,35 +188,38 @@ __device__ __forceinline__ int mla_half_tokens(int ctx, int j, int half) {
 // barrier slots.  Local: each CTA waits on its own.  Pair: live in the rank-0
 // CTA only (arrivals from both CTAs); the same slots are unused in the other.
 enum MlaBar {
-  kLatEmpty = 0,    // [2] local: the value MMA of the stage's tile is done (commit to both)
-  kSFull = 2,       // [2] local: scores of tile n in buffer n%2 (commit to both)
-  kOReady = 4,      // [2] local: value MMA of tile n done (commit to both; one slot per
-                    //     parity so that a waiter is never two phases behind)
-  kPvFull = 6,      // [2] local: the other CTA's tokens landed in this CTA's value slabs
-  kQEmpty = 8,      // local: last score MMA of a sequence done (commit to both)
-  kFinal = 9,       // local: every MMA done (commit to both)
-  kStall = 10,      // local, test hook only: nothing ever arrives here
-  kLatFull = 11,    // [2] pair: both CTAs' own tokens landed (2 arrivals + bytes)
-  kPhiFull = 13,    // pair: P hi of the tile written, its value rows in place (8 warps)
-  kQFull = 14,      // pair: query of a sequence in place in both CTAs (8 warps + 2 copies)
-  kOFree = 15,      // pair: both epilogues have read the accumulator (8 warps)
-  kPloFull = 16     // pair: P lo of the tile written in both CTAs (8 warps)
+  kLatEmpty = 0,    // [3] local: the value MMA of the stage's tile is done (commit to both)
+  kSFull = 3,       // [2] local: scores of tile n in the score buffer, slot n % 2 (commit
+                    //     to both; one slot per parity so that no waiter is two phases behind)
+  kOReady = 5,      // [2] local: value MMA of tile n done (commit to both, slot n % 2)
+  kPvFull = 7,      // [3] local: the other CTA's tokens landed in this CTA's value slabs
+  kQEmpty = 10,     // local: last score MMA of a sequence done (commit to both)
+  kFinal = 11,      // local: every MMA done (commit to both)
+  kStall = 12,      // local, test hook only: nothing ever arrives here
+  kPhiFree = 13,    // local: the P hi pass of the value MMA is done (commit to both)
+  kLatFull = 14,    // [3] pair: both CTAs' own tokens landed (2 arrivals + bytes)
+  kPhiFull = 17,    // pair: P hi of the tile written, its value rows in place (16 warps)
+  kQFull = 18,      // pair: query of a sequence in place in both CTAs (16 warps + 2 copies)
+  kOFree = 19,      // pair: both epilogues have read the accumulator (16 warps)
+  kPloFull = 20,    // pair: P lo of the tile written in both CTAs (16 warps)
+  kSFree = 21       // [2] pair: both CTAs' softmax warps have read score buffer n % 2 (16 warps)
 };
 
 __global__ void __launch_bounds__(kMlaThreads, 1)
-mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a32,
+                  const __grid_constant__ CUtensorMap tm_w9, const __grid_constant__ CUtensorMap tm_w2,
                   const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
   using L = MlaLayout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::bars);
-  float *xm = reinterpret_cast<float *>(sm + L::xch);            // [2][128] row maxima
-  float *xl = xm + 2 * 128;                                        // [128] row sums
+  float *xm = reinterpret_cast<float *>(sm + L::xch);            // [2][2][128] row maxima
+  float *xl = xm + 4 * 128;                                        // [2][128] row sums
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(sm + L::misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::misc + 4);
-  int *scan_scratch = reinterpret_cast<int *>(sm + L::misc + 16);   // [6]
-  int *start = reinterpret_cast<int *>(sm + L::misc + 48);          // b, j of the first tile
+  int *scan_scratch = reinterpret_cast<int *>(sm + L::misc + 16);   // [kMlaThreads / 32]
+  int *start = reinterpret_cast<int *>(sm + L::misc + 64);          // b, j of the first tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = pair::rank();        // 0: issues the MMAs; heads [64 rank, +64)
@@ -247,15 +271,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   if (tid == 0) {
     for (int i = 0; i < L::nbars; ++i) {
       uint32_t cnt = 1;
-      if (i == kLatFull || i == kLatFull + 1) cnt = 2;
-      if (i == kPhiFull || i == kPloFull || i == kOFree) cnt = 8;
-      if (i == kQFull) cnt = 10;          // 8 warps + each CTA's query copy (with its bytes)
+      if (i >= kLatFull && i < kLatFull + kMlaStages) cnt = 2;
+      if (i == kPhiFull || i == kPloFull || i == kOFree || i == kSFree || i == kSFree + 1)
+        cnt = 2 * kMlaSoftmaxWarps;
+      if (i == kQFull) cnt = 2 * kMlaSoftmaxWarps + 2;   // + each CTA's query copy (with its bytes)
       mbar_init(&bar[i], cnt);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMlaIssuer) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                      smem_u32(tmem_base_s))
                  : "memory");
@@ -279,6 +304,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   const int b_first = start[0], j_first = start[1];
   // the pair barriers, addressed in the rank-0 CTA
   const uint32_t phifull_pair = pair::map_to(&bar[kPhiFull], 0);
+  const uint32_t sfree_pair0 = pair::map_to(&bar[kSFree], 0);
+  const uint32_t sfree_pair1 = pair::map_to(&bar[kSFree + 1], 0);
   const uint32_t plofull_pair = pair::map_to(&bar[kPloFull], 0);
   const uint32_t qfull_pair = pair::map_to(&bar[kQFull], 0);
   const uint32_t ofree_pair = pair::map_to(&bar[kOFree], 0);
@@ -286,12 +313,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   // tokens for them are staged in the slabs of the same index xor 2
   const int vs0 = 2 * static_cast<int>(rank);
 
-  if (warp == 4) {
+  if (warp == kMlaProducer) {
     // ------------------------------------------------------------ copy issue
-    // Lane i holds the cache rows of the four 32-token boxes of tile wb + i
+    // Lane i holds the cache rows of the six 16-token boxes of tile wb + i
     // (current window) and wb + 32 + i (next window); lane 0 issues, whichever of
     // "own tokens of tile n" (stage free) and "other tokens of tile n" (scores of
-    // tile n done) is ready first.
+    // tile n done) is ready first.  A box is 16 rows x 64 dims (2 KB) of one slab.
     const uint64_t pol_keep = l2_evict_last_policy();
     const uint64_t pol_once = l2_evict_first_policy();
     bool aborted = false;
@@ -306,16 +333,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     }
     if (lane == 0) {
       prefetch_tensormap(&tm_a);
-      if (p.wide) prefetch_tensormap(&tm_b);
+      prefetch_tensormap(&tm_a32);
+      prefetch_tensormap(&tm_w9);
+      prefetch_tensormap(&tm_w2);
     }
+    // Copies of a CTA half (48 rows, the three 16-row groups at cache rows r[0..2],
+    // -2 for a group past the context): a run of 48 contiguous rows (the half lies
+    // in one block) moves as one 3-D box that lands as whole slabs; otherwise each
+    // run of 32 or 16 contiguous rows moves as one 2-D box per slab.  The copy
+    // engine takes about 17 boxes per microsecond per SM whatever their size, so
+    // the box count, not the bytes, bounds small copies.
+    auto run_of = [&](const int (&r)[kMlaBoxes], int k) {   // rows of the run starting at group k
+      if (k == 0 && r[1] == r[0] + kMlaBox && r[2] == r[0] + 2 * kMlaBox) return 3;
+      if (k < kMlaBoxes - 1 && r[k + 1] == r[k] + kMlaBox) return 2;
+      return 1;
+    };
     MlaCursor cur;
     cur.init(p, b_first, j_first, ntiles);
-    // Cache rows of the tile's boxes held by this lane: this CTA's two (own) and
-    // the other CTA's two (oth), for the current window (c*) and the next (n*)
-    const int own_box = 2 * static_cast<int>(rank), oth_box = 2 - own_box;
-    int c_own0 = -2, c_own1 = -2, c_oth0 = -2, c_oth1 = -2;
-    int n_own0 = -2, n_own1 = -2, n_oth0 = -2, n_oth1 = -2;
-    auto look_up = [&](int base, int &o0, int &o1, int &t0, int &t1) {
+    // Cache rows of the tile's boxes held by this lane: this CTA's three (own, c/n
+    // o*) and the other CTA's three (t*), for the current window (c) and the next (n)
+    const int own_box = kMlaBoxes * static_cast<int>(rank), oth_box = kMlaBoxes - own_box;
+    int c_o[kMlaBoxes], c_t[kMlaBoxes], n_o[kMlaBoxes], n_t[kMlaBoxes];
+#pragma unroll
+    for (int k = 0; k < kMlaBoxes; ++k) c_o[k] = c_t[k] = n_o[k] = n_t[k] = -2;
+    auto look_up = [&](int base, int (&o)[kMlaBoxes], int (&t)[kMlaBoxes]) {
       const int n = min(32, ntiles - base);
       int mb = 0, mj = 0, mctx = 0;
       for (int i = 0; i < n; ++i, cur.next())
@@ -325,20 +366,23 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           mctx = cur.ctx;
         }
       const bool ok = lane < n;
-      o0 = ok ? mla_box_row(p, mb, mj, own_box, mctx) : -2;
-      o1 = ok ? mla_box_row(p, mb, mj, own_box + 1, mctx) : -2;
-      t0 = ok ? mla_box_row(p, mb, mj, oth_box, mctx) : -2;
-      t1 = ok ? mla_box_row(p, mb, mj, oth_box + 1, mctx) : -2;
+#pragma unroll
+      for (int k = 0; k < kMlaBoxes; ++k) {
+        o[k] = ok ? mla_box_row(p, mb, mj, own_box + k, mctx) : -2;
+        t[k] = ok ? mla_box_row(p, mb, mj, oth_box + k, mctx) : -2;
+      }
     };
     int wb = 0;                      // first tile of the current window
-    if (ntiles > 0) look_up(0, c_own0, c_own1, c_oth0, c_oth1);
-    if (ntiles > 32) look_up(32, n_own0, n_own1, n_oth0, n_oth1);
-    // rows of tile n (all lanes call): k = 0, 1 own boxes, 2, 3 the other CTA's
-    auto row_of = [&](int n, int k) {
+    if (ntiles > 0) look_up(0, c_o, c_t);
+    if (ntiles > 32) look_up(32, n_o, n_t);
+    // rows of tile n's boxes (all lanes call): own (oth = false) or the other CTA's
+    auto rows_of = [&](int n, bool oth, int (&r)[kMlaBoxes]) {
       const bool w = n - wb >= 32;
-      const int v = k == 0 ? (w ? n_own0 : c_own0) : k == 1 ? (w ? n_own1 : c_own1)
-                  : k == 2 ? (w ? n_oth0 : c_oth0) : (w ? n_oth1 : c_oth1);
-      return __shfl_sync(0xffffffffu, v, (n - wb) & 31);
+#pragma unroll
+      for (int k = 0; k < kMlaBoxes; ++k) {
+        const int v = oth ? (w ? n_t[k] : c_t[k]) : (w ? n_o[k] : c_o[k]);
+        r[k] = __shfl_sync(0xffffffffu, v, (n - wb) & 31);
+      }
     };
     int n_own = 0, n_pv = 0;
     uint64_t t_idle = globaltimer();
@@ -346,88 +390,103 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     while (n_pv < ntiles && !aborted) {
       // slide the windows once the other-token loads have left the current one
       if (n_pv >= wb + 32) {
-        c_own0 = n_own0;
-        c_own1 = n_own1;
-        c_oth0 = n_oth0;
-        c_oth1 = n_oth1;
+#pragma unroll
+        for (int k = 0; k < kMlaBoxes; ++k) {
+          c_o[k] = n_o[k];
+          c_t[k] = n_t[k];
+        }
         wb += 32;
-        if (ntiles > wb + 32) look_up(wb + 32, n_own0, n_own1, n_oth0, n_oth1);
+        if (ntiles > wb + 32) look_up(wb + 32, n_o, n_t);
       }
       int act = 0;
       if (lane == 0) {
-        if (n_own < ntiles && n_own < n_pv + kMlaStages &&
+        // own tokens run at most one tile ahead of the next other-token fetch: the
+        // fetch (an L2 hit that the value MMA waits on) queues behind this SM's
+        // copies in flight, so fewer of them ahead of it means a shorter wait
+        if (n_own < ntiles && n_own < n_pv + kMlaLookahead &&
             (n_own < kMlaStages ||
              mbar_test(&bar[kLatEmpty + n_own % kMlaStages], ((n_own / kMlaStages) & 1) ^ 1)))
           act = 1;
-        else if (n_pv < n_own &&
-                 mbar_test(&bar[kSFull + n_pv % kMlaStages], (n_pv / kMlaStages) & 1))
-          act = 2;
+        if (n_pv < n_own && mbar_test(&bar[kSFull + n_pv % 2], (n_pv / 2) & 1))
+          act = 2;                       // the other CTA's tokens first: the value MMA waits on them
       }
       act = __shfl_sync(0xffffffffu, act, 0);
       if (act == 1) {
         const int n = n_own++;
         const int st = n % kMlaStages;
-        const int r0 = row_of(n, 0), r1 = row_of(n, 1);
-        // the own tokens of the tile that next uses this stage, pulled into L2 now
-        // (one copy instruction): their load, issued once this tile's value MMA is
-        // done, then finds them in L2
-        const int f0 = p.wide && n + kMlaStages < ntiles ? row_of(n + kMlaStages, 0) : -2;
+        int r[kMlaBoxes];
+        rows_of(n, false, r);
         if (lane == 0) {
-          if (f0 >= 0) tma_prefetch_3d(&tm_a, 0, f0, 0, pol_keep);
-          if (r0 == -1 || r1 == -1) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
-          const uint32_t bytes =
-              p.wide ? (r0 >= 0 ? L::kStage : 0)
-                     : L::kSlabs * kMlaBox * 128 * ((r0 >= 0) + (r1 >= 0));
-          const uint32_t full = pair::map_to(&bar[kLatFull + st], 0);
-          pair::arrive_expect_tx_remote(full, bytes);
-          uint8_t *dst = sm + L::stage + st * L::kStage;
-          if (p.wide) {
-            // the 64 tokens in one copy: a 64 dims x 64 rows x 9 slabs box lands as
-            // the stage's 9 slabs (r1 is r0's second half, or past the context)
-            if (r0 >= 0) pair::tma_load_3d_to_pair_bar(dst, &tm_a, full, 0, r0, 0, pol_keep);
-          } else {
-#pragma unroll 1
-            for (int s = 0; s < L::kSlabs; ++s) {
-              if (r0 >= 0)
-                pair::tma_load_2d_to_pair_bar(dst + s * L::kSlab, &tm_a, full, 64 * s, r0,
-                                              pol_keep);
-              if (r1 >= 0)
-                pair::tma_load_2d_to_pair_bar(dst + s * L::kSlab + kMlaBox * 128, &tm_a, full,
-                                              64 * s, r1, pol_keep);
-            }
+          int boxes = 0;
+#pragma unroll
+          for (int k = 0; k < kMlaBoxes; ++k) {
+            if (r[k] == -1) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
+            boxes += r[k] >= 0;
           }
+          const uint32_t full = pair::map_to(&bar[kLatFull + st], 0);
+          pair::arrive_expect_tx_remote(full, L::kSlabs * kMlaBox * 128 * boxes);
+          uint8_t *dst = sm + L::stage + st * L::kStage;
+          for (int k = 0; k < kMlaBoxes;) {
+            const int len = r[k] >= 0 ? run_of(r, k) : 1;
+            if (r[k] >= 0 && len == 3) {
+              pair::tma_load_3d_to_pair_bar(dst, &tm_w9, full, 0, r[k], 0, pol_keep);
+            } else if (r[k] >= 0) {
+#pragma unroll 1
+              for (int sl = 0; sl < L::kSlabs; ++sl)
+                pair::tma_load_2d_to_pair_bar(dst + sl * L::kSlab + k * kMlaBox * 128,
+                                              len == 2 ? &tm_a32 : &tm_a, full, 64 * sl, r[k],
+                                              pol_keep);
+            }
+            k += len;
+          }
+        }
+        // Pull the own rows of the tile kMlaPrefetch ahead into L2 (kept there): its
+        // copy, issued once a stage frees, then reads L2 instead of waiting on HBM
+        // behind this SM's other copies.  One bulk prefetch per contiguous run.
+        if (kMlaPrefetch > 0 && n + kMlaPrefetch < ntiles) {
+          int f[kMlaBoxes];
+          rows_of(n + kMlaPrefetch, false, f);
+          if (lane == 0)
+            for (int k = 0; k < kMlaBoxes;) {
+              const int len = f[k] >= 0 ? run_of(f, k) : 1;
+              if (f[k] >= 0)
+                prefetch_l2_bulk(p.lat + static_cast<long long>(f[k]) * kMlaDk,
+                                 len * kMlaBox * kMlaDk * 2, pol_keep);
+              k += len;
+            }
         }
       } else if (act == 2) {
         const int n = n_pv++;
         const int st = n % kMlaStages;
-        const int r0 = row_of(n, 2), r1 = row_of(n, 3);
+        int r[kMlaBoxes];
+        rows_of(n, true, r);
         if (lane == 0) {
-          const uint32_t bytes = p.wide ? (r0 >= 0 ? 4 * L::kSlab : 0)
-                                        : 4 * kMlaBox * 128 * ((r0 >= 0) + (r1 >= 0));
-          mbar_arrive_expect_tx(&bar[kPvFull + st], bytes);
+          int boxes = 0;
+#pragma unroll
+          for (int k = 0; k < kMlaBoxes; ++k) boxes += r[k] >= 0;
+          mbar_arrive_expect_tx(&bar[kPvFull + st], 4 * kMlaBox * 128 * boxes);
           // the value dims: latent slabs vs0, vs0 + 1, vs0 + 4, vs0 + 5, into the
           // stage's slabs of index xor 2
           uint8_t *dst = sm + L::stage + st * L::kStage;
-          if (p.wide) {
-            // two 64 dims x 64 rows x 2 slabs boxes
+          for (int k = 0; k < kMlaBoxes;) {
+            const int len = r[k] >= 0 ? run_of(r, k) : 1;
+            if (r[k] >= 0 && len == 3) {
+              // two 64 dims x 48 rows x 2 slabs boxes (slab pairs vs0, vs0 + 1 and
+              // vs0 + 4, vs0 + 5 into the pairs of index xor 2)
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const int sl = vs0 + 4 * g;
-              if (r0 >= 0)
-                tma_load_3d_hint(dst + (sl ^ 2) * L::kSlab, &tm_b, &bar[kPvFull + st], 0, r0, sl,
-                                 pol_once);
-            }
-          } else {
+              for (int g = 0; g < 2; ++g)
+                tma_load_3d_hint(dst + ((vs0 + 4 * g) ^ 2) * L::kSlab, &tm_w2, &bar[kPvFull + st],
+                                 0, r[k], vs0 + 4 * g, pol_once);
+            } else if (r[k] >= 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int sl = vs0 + (i & 1) + 4 * (i >> 1);
-              if (r0 >= 0)
-                tma_load_2d_hint(dst + (sl ^ 2) * L::kSlab, &tm_a, &bar[kPvFull + st], 64 * sl, r0,
+              for (int i = 0; i < 4; ++i) {
+                const int sl = vs0 + (i & 1) + 4 * (i >> 1);
+                tma_load_2d_hint(dst + (sl ^ 2) * L::kSlab + k * kMlaBox * 128,
+                                 len == 2 ? &tm_a32 : &tm_a, &bar[kPvFull + st], 64 * sl, r[k],
                                  pol_once);
-              if (r1 >= 0)
-                tma_load_2d_hint(dst + (sl ^ 2) * L::kSlab + kMlaBox * 128, &tm_a,
-                                 &bar[kPvFull + st], 64 * sl, r1, pol_once);
+              }
             }
+            k += len;
           }
         }
       }
@@ -457,7 +516,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const uint64_t t0 = globaltimer();
       while (globaltimer() - t0 < 50000) __nanosleep(1000);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMlaIssuer) {
     // ------------------------------------------------------------ MMA issuer (rank 0)
     if (rank == 0 && lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, kMlaTile, false);
@@ -468,7 +527,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const uint64_t v_desc0 = umma_desc(smem_u32(sm + L::stage), L::kSlab, 1024);  // MN-major
       const uint64_t q_desc0 = umma_desc(smem_u32(sm + L::qs), 16, 1024);
       const uint64_t p_desc0 = umma_desc(smem_u32(sm + L::ps), 16, 1024);
-      const uint64_t pst_desc0 = umma_desc(smem_u32(sm + L::stage), 16, 1024);  // K-major P
       int s_seg = -1, o_seg = -1;
       MlaCursor cs, cp;                  // tile walks of the score and value MMAs
       cs.init(p, b_first, j_first, ntiles);
@@ -481,8 +539,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (first) ++s_seg;
         tc_fence_after();
         const uint64_t bst = b_desc0 + ((st * L::kStage) >> 4);
-        const uint32_t d = tmem + kTmS + (n % 2) * (kMlaTile / 2);
-        // 16-dim step ks reads latent slab ks/4 at byte offset 32 (ks%4) of each row
+        const uint32_t d = tmem + kTmS + (n % 2) * kMlaHalf;
+        // 16-dim step ks reads latent slab ks/4 at byte offset 32 (ks%4) of each row;
+        // the query's first 320 dims come from tensor memory, the rest from its
+        // shared-memory slabs
 #pragma unroll
         for (int ks = 0; ks < kMlaDk / 16; ++ks) {
           const uint64_t b = bst + (((ks >> 2) * L::kSlab + (ks & 3) * 32) >> 4);
@@ -490,7 +550,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             pair::mma_ts(d, tmem + kTmQ + ks * 8, b, idesc_s, ks > 0);
           } else {
             const int kq = ks - kQTmemDims / 16;
-            pair::mma_ss(d, q_desc0 + (((kq >> 2) * L::kSlab + (kq & 3) * 32) >> 4), b, idesc_s,
+            pair::mma_ss(d, q_desc0 + (((kq >> 2) * L::kHSlab + (kq & 3) * 32) >> 4), b, idesc_s,
                          true);
           }
         }
@@ -498,11 +558,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (last) pair::commit_both(&bar[kQEmpty]);
       };
       // The value MMA of tile n in two passes: P hi (written as soon as the softmax
-      // is done), then P lo (whose single buffer the previous tile's lo pass must
-      // have released).  Dims block nb: the CTAs supply dims [256nb, 256nb+128)
+      // is done), then P lo.  Dims block nb: the CTAs supply dims [256nb, 256nb+128)
       // and [256nb+128, 256nb+256); token half h of the tile sits in slabs
       // 4nb + 2h, 4nb + 2h + 1 of both CTAs (own tokens or the other CTA's, see
-      // above); 16 tokens (2 KB) per step.
+      // above); 16 tokens (2 KB of each slab) per step.  P's 16 tokens from t0 on
+      // lie in pool slab 0 (hi) or 2 (lo) for t0 < 64, else in slab 1 (hi in the
+      // first 64 bytes of a row, lo in the last 64).
       auto issue_pv = [&](int n, bool lo_pass) {
         const int st = n % kMlaStages;
         bool first = false;
@@ -518,14 +579,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           for (int h = 0; h < 2; ++h) {
             const uint64_t vb = v_desc0 + ((st * L::kStage + (4 * nb + 2 * h) * L::kSlab) >> 4);
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-              uint64_t a;
-              if (lo_pass)
-                a = p_desc0 + (((2 + h) * L::kSlab + kq * 32) >> 4);
-              else if (h == 0)
-                a = pst_desc0 + ((st * L::kStage + 8 * L::kSlab + kq * 32) >> 4);
-              else
-                a = p_desc0 + (((n & 1) * L::kSlab + kq * 32) >> 4);
+            for (int kq = 0; kq < kMlaBoxes; ++kq) {
+              const int t0 = kMlaHalf * h + 16 * kq;
+              const int poff = t0 < 64 ? (lo_pass ? 2 : 0) * L::kHSlab + 2 * t0
+                                       : L::kHSlab + (lo_pass ? 64 : 0) + 2 * (t0 - 64);
+              const uint64_t a = p_desc0 + (poff >> 4);
               const uint64_t b = vb + ((kq * 2048) >> 4);
               pair::mma_ss(tmem + kTmO + nb * 128, a, b, idesc_o,
                            lo_pass || !(first && h == 0 && kq == 0));
@@ -535,21 +593,23 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (lo_pass) {
           pair::commit_both(&bar[kLatEmpty + st]);
           pair::commit_both(&bar[kOReady + n % 2]);
+        } else {
+          pair::commit_both(&bar[kPhiFree]);
         }
       };
       // S(m), PVhi(m) and PVlo(m) are each issued in tile order, whichever is ready
-      // first: S(m) once PVhi(m-2) is issued (it reuses that score buffer, which
-      // the softmax had read before writing P hi; the tensor pipe runs one
-      // thread's MMAs in order), both CTAs' own tokens of tile m have landed and,
-      // at a sequence start, the query is in place; PVhi(m) once P hi is written
-      // and the value rows are in place in both CTAs and, at a sequence start, the
-      // previous O has been read out; PVlo(m) once P lo is written.
+      // first: S(m) once both CTAs' softmax warps have read S(m-2) out of score
+      // buffer m % 2, both CTAs' own tokens of tile m have landed and, at a sequence
+      // start, the query is in place; PVhi(m) once P hi is written and the value
+      // rows are in place in both CTAs and, at a sequence start, the previous O
+      // has been read out; PVlo(m) once P lo is written.
       int ns = 0, nh = 0, nl = 0;
       uint64_t t_idle = globaltimer();
       uint32_t spins = 0;
       while (nl < ntiles) {
         bool did = false;
-        if (ns < ntiles && ns < nh + 2 &&
+        if (ns < ntiles &&
+            (ns < 2 || pair::test_cluster(&bar[kSFree + ns % 2], ((ns / 2) & 1) ^ 1)) &&
             pair::test_cluster(&bar[kLatFull + ns % kMlaStages], (ns / kMlaStages) & 1) &&
             (!cs.first() || pair::test_cluster(&bar[kQFull], (s_seg + 1) & 1))) {
           issue_s(ns++);
@@ -581,23 +641,33 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     if (rank == 0 && lane == 0) pair::commit_both(&bar[kFinal]);
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax / epilogue (warps 0-3)
-    const int t = tid;                                 // TMEM lane
-    const int lh = t & 63;                             // head 64 rank + lh
-    const int hh = t >> 6;                             // token half of each tile
+    // ------------------------------------------------------------ softmax / epilogue (warps 0-7)
+    // Warp w reads TMEM lanes [32 (w % 4), +32) (the lanes a warp may access) and
+    // column group cg = w / 4 of them.  A head's row of scores lies in lanes l and
+    // 64 + l (token halves), and each lane's 48 columns are split between the two
+    // column groups: cg 0 takes columns [0, 16) and [32, 40), cg 1 [16, 32) and
+    // [40, 48) (loads of 16 and 8 columns at offsets aligned to their size).  So
+    // four threads share a head: (hh, cg), in warps w, w + 2, w + 4, w + 6.
+    const int t = tid;
+    const int cg = warp >> 2;                          // column group
+    const int tl = 32 * (warp & 3) + lane;             // TMEM lane
+    const int lh = tl & 63;                            // head 64 rank + lh
+    const int hh = tl >> 6;                            // token half of each tile
     const int head = 64 * static_cast<int>(rank) + lh;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    // the thread's tokens: 8-token chunks {2 cg, 2 cg + 1, 4 + cg} of its half
+    auto chunk_of = [&](int i) { return i < 2 ? 2 * cg + i : 4 + cg; };
     bool aborted = false;
 
-    // Query of sequence b.  Dims [256, 576) of the CTA's 64 heads land in shared
-    // memory with one copy (a 64 dims x 64 rows x 5 slabs box: the 128-byte
+    // Query of sequence b.  Dims [320, 576) of the CTA's 64 heads land in shared
+    // memory with one copy (a 64 dims x 64 rows x 4 slabs box: the 128-byte
     // swizzled K-major layout of the A operand), counted on the rank-0 CTA's
-    // query barrier.  Dims [0, 256) go into TMEM lane t as bf16 pairs (both lanes
-    // of the head: the layout of a 2-SM A operand), loaded in two batches of 128
+    // query barrier.  Dims [0, 320) go into TMEM lane t as bf16 pairs (both lanes
+    // of the head: the layout of a 2-SM A operand), loaded in five batches of 64
     // dims.  Called after the previous sequence's last score MMA.
     auto load_query = [&](int b) {
       if (t == 0) {
-        pair::arrive_expect_tx_remote(qfull_pair, L::kQSlabs * L::kSlab);
+        pair::arrive_expect_tx_remote(qfull_pair, L::kQSlabs * L::kHSlab);
         pair::tma_load_3d_to_pair_bar(sm + L::qs, &tm_q, qfull_pair, 0,
                                       b * kMlaHeads + 64 * static_cast<int>(rank),
                                       kQTmemDims / 64, l2_evict_first_policy());
@@ -605,22 +675,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const uint4 *src = reinterpret_cast<const uint4 *>(
           p.q + (static_cast<long long>(b) * kMlaHeads + head) * kMlaDk);
 #pragma unroll 1
-      for (int g = 0; g < kQTmemDims / 64; g += 2) {
-        uint4 x[16];
+      for (int g = cg == 0 ? 0 : 3; g < (cg == 0 ? 3 : kQTmemDims / 64); ++g) {
+        uint4 x[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = __ldg(src + g * 8 + i);
+        for (int i = 0; i < 8; ++i) x[i] = __ldg(src + g * 8 + i);
+        uint32_t v[32];
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          uint32_t v[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[4 * i] = x[8 * k + i].x;
-            v[4 * i + 1] = x[8 * k + i].y;
-            v[4 * i + 2] = x[8 * k + i].z;
-            v[4 * i + 3] = x[8 * k + i].w;
-          }
-          tmem_st32u(tmem + kTmQ + (g + k) * 32 + lane_off, v);
+        for (int i = 0; i < 8; ++i) {
+          v[4 * i] = x[i].x;
+          v[4 * i + 1] = x[i].y;
+          v[4 * i + 2] = x[i].z;
+          v[4 * i + 3] = x[i].w;
         }
+        tmem_st32u(tmem + kTmQ + g * 32 + lane_off, v);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -630,26 +697,27 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 
     // Pull the query of sequence b into L2 a tile ahead of load_query, marked to
     // stay (the latent tiles streaming meanwhile are marked the same way): the
-    // TMEM part (dims [0, 256): four 128-byte lines, two per thread of the head)
+    // TMEM part (dims [0, 320): five 128-byte lines, shared by the head's two
+    // threads)
     // and the shared-memory part's box.
     const uint64_t pol_q = l2_evict_last_policy();
     auto prefetch_query = [&](int b) {
       if (b < 0 || b >= p.B) return;
       const char *row = reinterpret_cast<const char *>(
           p.q + (static_cast<long long>(b) * kMlaHeads + head) * kMlaDk);
-      for (int i = hh; i < kQTmemDims * 2 / 128; i += 2)
+      for (int i = hh + 2 * cg; i < kQTmemDims * 2 / 128; i += 4)
         asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(row + i * 128));
       if (t == 0)
         tma_prefetch_3d(&tm_q, 0, b * kMlaHeads + 64 * static_cast<int>(rank), kQTmemDims / 64,
                         pol_q);
     };
 
-    // Zero rows [from, 64) of the four slabs at slab indices first, first + 1,
+    // Zero rows [from, 48) of the four slabs at slab indices first, first + 1,
     // first + 4, first + 5 of a stage (value rows of tokens past a ragged end, so
-    // that 0 x stale data stays 0); the 128 threads share the work.
+    // that 0 x stale data stays 0); the softmax threads share the work.
     auto zero_rows = [&](uint8_t *stage, int first, int from) {
       const int rows = kMlaHalf - from;
-      for (int i = t; i < rows * 4 * 8; i += 128) {
+      for (int i = t; i < rows * 4 * 8; i += 32 * kMlaSoftmaxWarps) {
         const int sl = first + (i / (rows * 8) & 1) + 4 * ((i / (rows * 8)) >> 1);
         const int r = from + (i / 8) % rows, ch = i % 8;
         *reinterpret_cast<uint4 *>(stage + sl * L::kSlab + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
@@ -695,28 +763,36 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const int st = n % kMlaStages;
       uint8_t *stage = sm + L::stage + st * L::kStage;
       const int ntok = mla_half_tokens(ctx, j, hh);
-      float sc[kMlaHalf];
+      float sc[kMlaTok];
       {
         const bool got = !aborted && mbar_wait(&bar[kSFull + n % 2], (n / 2) & 1, abort_flag);
         aborted = !__all_sync(0xffffffffu, got);
         tc_fence_after();
-        const uint32_t scol = tmem + kTmS + (n % 2) * (kMlaTile / 2) + lane_off;
-        float (&s0)[32] = *reinterpret_cast<float (*)[32]>(&sc[0]);
-        float (&s1)[32] = *reinterpret_cast<float (*)[32]>(&sc[32]);
-        tmem_ld32(scol, s0);
-        tmem_ld32(scol + 32, s1);
+        const uint32_t scol = tmem + kTmS + (n % 2) * kMlaHalf + lane_off;
+        float (&s0)[16] = *reinterpret_cast<float (*)[16]>(&sc[0]);
+        float (&s1)[8] = *reinterpret_cast<float (*)[8]>(&sc[16]);
+        tmem_ld16(scol + 16 * cg, s0);
+        tmem_ld8(scol + 32 + 8 * cg, s1);
         tmem_wait_ld();
+        // the score buffer is free for the next tile's score MMA
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) pair::arrive_remote(n % 2 ? sfree_pair1 : sfree_pair0);
       }
-      // ---- online softmax (log2 units); the head's two threads agree on the max
+      // ---- online softmax (log2 units); the head's four threads agree on the max
       float mt = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < kMlaHalf; ++i) {
-        sc[i] = i < ntok ? sc[i] * p.scale_log2 : -INFINITY;
+      for (int i = 0; i < kMlaTok; ++i) {
+        sc[i] = 8 * chunk_of(i / 8) + i % 8 < ntok ? sc[i] * p.scale_log2 : -INFINITY;
         mt = fmaxf(mt, sc[i]);
       }
-      xm[(n & 1) * 128 + t] = mt;
-      named_bar_sync(1 + (warp & 1), 64);      // warps w and w + 2 hold the same heads
-      mt = fmaxf(mt, xm[(n & 1) * 128 + (t ^ 64)]);
+      {
+        float *x = xm + (n & 1) * 256;
+        x[cg * 128 + tl] = mt;
+        named_bar_sync(1 + (warp & 1), 128);   // warps w, w + 2, w + 4, w + 6 hold the same heads
+        mt = fmaxf(fmaxf(mt, x[cg * 128 + (tl ^ 64)]),
+                   fmaxf(x[(1 - cg) * 128 + tl], x[(1 - cg) * 128 + (tl ^ 64)]));
+      }
       const bool raise = mt > m_run + kMlaRescale;
       bool pv_prev_done = n == 0;
       if (__any_sync(0xffffffffu, raise && !first)) {
@@ -728,7 +804,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         tc_fence_after();
         pv_prev_done = true;
         const float alpha = (raise && !first) ? ex2_approx(m_run - mt) : 1.f;
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 128 * cg; c < 128 * cg + 128; c += 32) {
           float v[32];
           tmem_ld32(tmem + kTmO + c + lane_off, v);
           tmem_wait_ld();
@@ -742,26 +818,33 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       }
       if (raise) m_run = mt;
       // ---- P = 2^(s - m) as a bf16 hi + lo pair, into this thread's row of the
-      // A operand of the value MMA: heads x 128 tokens, K-major, 128-byte swizzle
-      // (token half hh = slab hh; hi slabs first, lo slabs 16 KB on)
-      uint32_t hi[32], lo[32];
+      // A operand of the value MMA: heads x 96 tokens, K-major, 128-byte swizzle;
+      // 16-byte chunk c of a row holds tokens 48 hh + 8c .. + 7 (pool slabs: see
+      // the layout), and this thread writes chunks chunk_of(0..2)
+      uint32_t hi[kMlaTok / 2], lo[kMlaTok / 2];
 #pragma unroll
-      for (int e = 0; e < kMlaHalf / 2; ++e) {
+      for (int e = 0; e < kMlaTok / 2; ++e) {
         const float p0 = ex2_approx(sc[2 * e] - m_run);
         const float p1 = ex2_approx(sc[2 * e + 1] - m_run);
         split2<true>(p0, p1, hi[e], lo[e]);
         l_run += p0 + p1;
       }
-      {
-        // P hi: token half 0 into slab 8 of the tile's stage, half 1 into the pool
-        // slab of this tile's parity (both free: see the layout)
-        uint8_t *prow = hh == 0 ? stage + 8 * L::kSlab + lh * 128
-                                : sm + L::ps + (n & 1) * L::kSlab + lh * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(prow + ((c ^ (lh & 7)) << 4)) =
-              make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+      // where chunk c of P goes: pool slab and 16-byte column of row lh
+      auto p_chunk = [&](int c, bool lo_copy) {
+        const int tk = kMlaHalf * hh + 8 * c;
+        const int slab = tk < 64 ? (lo_copy ? 2 : 0) : 1;
+        const int col = tk < 64 ? tk / 8 : (lo_copy ? 4 : 0) + (tk - 64) / 8;
+        return sm + L::ps + slab * L::kHSlab + lh * 128 + ((col ^ (lh & 7)) << 4);
+      };
+      // P hi: its single buffer is released by the previous tile's hi pass
+      if (n > 0) {
+        const bool got = !aborted && mbar_wait(&bar[kPhiFree], (n - 1) & 1, abort_flag);
+        aborted = !__all_sync(0xffffffffu, got);
       }
+#pragma unroll
+      for (int c = 0; c < kMlaTok / 8; ++c)
+        *reinterpret_cast<uint4 *>(p_chunk(chunk_of(c), false)) =
+            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
       // ---- tokens past a ragged end: zero their value rows, own tokens now (the
       // scores are done with them), the other CTA's once they have landed
       const bool ragged = (j + 1) * kMlaTile > ctx;
@@ -787,13 +870,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                                                abort_flag);
         aborted = !__all_sync(0xffffffffu, got);
       }
-      {
-        uint8_t *prow = sm + L::ps + (2 + hh) * L::kSlab + lh * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(prow + ((c ^ (lh & 7)) << 4)) =
-              make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-      }
+      for (int c = 0; c < kMlaTok / 8; ++c)
+        *reinterpret_cast<uint4 *>(p_chunk(chunk_of(c), true)) =
+            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) pair::arrive_remote(plofull_pair);
@@ -806,15 +886,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         const bool got = !aborted && mbar_wait(&bar[kOReady + n % 2], (n / 2) & 1, abort_flag);
         aborted = !__all_sync(0xffffffffu, got);
         tc_fence_after();
-        xl[t] = l_run;
-        named_bar_sync(1 + (warp & 1), 64);
-        const float l_tot = l_run + xl[t ^ 64];
+        xl[cg * 128 + tl] = l_run;
+        named_bar_sync(1 + (warp & 1), 128);
+        const float l_tot = (l_run + xl[cg * 128 + (tl ^ 64)]) +
+                            (xl[(1 - cg) * 128 + tl] + xl[(1 - cg) * 128 + (tl ^ 64)]);
         // the sequence's tiles all lie in this piece iff it starts and ends inside
         const bool whole = n - j >= 0 && n - j + P <= ntiles;
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const long long slot = pc + b;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 128 * cg; c < 128 * cg + 128; c += 32) {
           float v[32];
           tmem_ld32(tmem + kTmO + c + lane_off, v);
           tmem_wait_ld();
@@ -840,7 +921,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                   v[4 * q4] * inv, v[4 * q4 + 1] * inv, v[4 * q4 + 2] * inv, v[4 * q4 + 3] * inv);
           }
         }
-        if (!whole && hh == 0)
+        if (!whole && hh == 0 && cg == 0)
           p.part_lse[slot * kMlaHeads + head] = l_tot > 0.f ? m_run + log2f(l_tot) : -INFINITY;
         tc_fence_before();
         __syncwarp();
@@ -852,7 +933,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   // ---- teardown: every MMA of the pair has completed before either CTA frees
   // its tensor memory, and neither CTA leaves while the other may still signal it
   __syncthreads();
-  if (warp == 5 && lane == 0) {
+  if (warp == kMlaIssuer && lane == 0) {
     volatile int never = 0;
     mbar_wait(&bar[kFinal], 0, &never);
   }
@@ -860,7 +941,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   __syncthreads();
   pair::cluster_sync();
   tc_fence_after();
-  if (warp == 5)
+  if (warp == kMlaIssuer)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
 }
 

@@ -81,7 +81,7 @@ def test_ragged_and_tiny_contexts(dev):
         assert torch.all(out[3] == 0)
 
 
-@pytest.mark.parametrize("bs", [32, 64, 128])
+@pytest.mark.parametrize("bs", [16, 32, 48, 64, 128])
 def test_block_sizes(dev, bs):
     inp = workloads.make(mla((200, 1000, 63), seed=3, bs=bs))
     ref = ref_of(inp)
