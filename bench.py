@@ -305,6 +305,24 @@ def parity_sample(w, inp, out_host, n=32, seed=0):
             "tolerance": "|out - oracle| <= 2e-3 + 1e-2 |oracle| elementwise (float64 oracle)"}
 
 
+def size_sample(run, cl, batch, target_s):
+    """Leading sequences of the batch that one oracle run covers in about target_s:
+    the sample grows from the first sequence, each estimate of the time per token
+    taken from the last run (a short first sequence alone overstates it), at least
+    doubling each time.  Returns the sequence count and the last run's seconds."""
+    nseq = 1
+    dt = run(nseq)
+    while nseq < batch and dt < 0.5 * target_s:
+        per_tok = max(dt, 1e-4) / max(int(cl[:nseq].sum()), 1)
+        k, acc = 0, 0.0
+        while k < batch and acc + per_tok * int(cl[k]) <= target_s:
+            acc += per_tok * int(cl[k])
+            k += 1
+        nseq = min(batch, max(k, 2 * nseq))
+        dt = run(nseq)
+    return nseq, dt
+
+
 def cpu_baseline(w, inp, target_s):
     """Time the float64 oracle on a bounded sample (leading sequences of the batch)."""
     import numpy as np
@@ -318,17 +336,10 @@ def cpu_baseline(w, inp, target_s):
         oracle_rows(w, inp, pairs, threads)
         return time.perf_counter() - t0
 
-    # calibrate on the first sequence (all heads), then grow to ~target_s; when the
-    # whole batch takes less than that, repeat whole passes until it is reached
-    t1 = max(run(1, H), 1e-4)
-    per_tok = t1 / max(int(cl[0]), 1)
-    nseq, acc = 0, 0.0
-    while nseq < w.batch and acc + per_tok * int(cl[nseq]) <= target_s:
-        acc += per_tok * int(cl[nseq])
-        nseq += 1
-    nseq = max(nseq, 1)
-    dt, reps = 0.0, 0
-    while reps == 0 or (nseq == w.batch and dt < target_s and reps < 1000):
+    # when the whole batch takes less than target_s, whole passes repeat until it is
+    nseq, dt = size_sample(lambda k: run(k, H), cl, w.batch, target_s)
+    reps = 1
+    while nseq == w.batch and dt < target_s and reps < 1000:
         dt += run(nseq, H)
         reps += 1
     sample_cl = cl[:nseq]
@@ -583,13 +594,7 @@ def run_reference(args, rank, world):
         oracle_rows(w, inp, pairs, nthreads)
         return time.perf_counter() - t0
 
-    t1 = max(step(1), 1e-4)
-    per_tok = t1 / max(int(cl[0]), 1)
-    nseq, acc = 0, 0.0
-    while nseq < w.batch and acc + per_tok * int(cl[nseq]) <= budget_per_step:
-        acc += per_tok * int(cl[nseq])
-        nseq += 1
-    nseq = max(nseq, 1)
+    nseq, _ = size_sample(step, cl, w.batch, budget_per_step)
     for _ in range(args.warmup):
         step(nseq)
     times = [step(nseq) for _ in range(args.steps)]
