@@ -48,7 +48,7 @@
 // Shared memory per CTA: three 54 KB latent stages, query dims [320, 576)
 // (32 KB), and P as a bf16 hi + lo pair (24 KB, the A operand of the value MMA).
 //
-// Warp roles (320 threads per CTA).  Warps 0-7 (four threads per head: token
+// Warp roles (352 threads per CTA).  Warps 0-7 (four threads per head: token
 // half hh and column group cg of each tile, 24 tokens each): query loads, the
 // online softmax in log2 units (a head's four threads agree on the running max
 // through shared memory, with a lazily raised max), P as bf16 hi + lo (about 16
@@ -56,8 +56,9 @@
 // weight), zeroing value rows past a ragged end, and the epilogue.  Warp 8
 // issues the TMA loads: its own tokens (completion counted on the rank-0 CTA's
 // barrier, so that the MMA issuer sees both halves land), and, once the tile's
-// scores are done, the other CTA's tokens for its value dims.  Warp 9 of the
-// rank-0 CTA issues every MMA from one thread.  Every wait is bounded.
+// scores are done, the other CTA's tokens for its value dims.  Warps 9 and 10 of
+// the rank-0 CTA issue the score and the value MMAs, one thread each.  Every wait
+// is bounded.
 #pragma once
 
 #include "pa_device.cuh"
@@ -83,8 +84,9 @@ constexpr int kMlaLookahead = PA_MLA_LOOKAHEAD;   // own-token tiles issued past
 constexpr int kMlaPrefetch = PA_MLA_PREFETCH;     // tiles ahead whose own rows are pulled into L2
 constexpr int kMlaSoftmaxWarps = 8;       // warps 0-7: softmax and epilogue
 constexpr int kMlaProducer = 8;           // warp 8: copy issue
-constexpr int kMlaIssuer = 9;             // warp 9: MMA issue (rank 0), TMEM allocation
-constexpr int kMlaThreads = 32 * (kMlaSoftmaxWarps + 2);
+constexpr int kMlaIssuer = 9;             // warp 9: score MMA issue (rank 0), TMEM allocation
+constexpr int kMlaPvIssuer = 10;          // warp 10: value MMA issue (rank 0)
+constexpr int kMlaThreads = 32 * (kMlaSoftmaxWarps + 3);
 constexpr int kMlaTok = kMlaHalf / 2;     // tokens of a tile per softmax thread
 constexpr int kMlaRescale = 8;            // raise the running max only past 2^8 growth
 
@@ -194,7 +196,7 @@ enum MlaBar {
   kOReady = 5,      // [2] local: value MMA of tile n done (commit to both, slot n % 2)
   kPvFull = 7,      // [3] local: the other CTA's tokens landed in this CTA's value slabs
   kQEmpty = 10,     // local: last score MMA of a sequence done (commit to both)
-  kFinal = 11,      // local: every MMA done (commit to both)
+  kFinal = 11,      // local: every MMA done (one commit to both from each issuer)
   kStall = 12,      // local, test hook only: nothing ever arrives here
   kPhiFree = 13,    // local: the P hi pass of the value MMA is done (commit to both)
   kLatFull = 14,    // [3] pair: both CTAs' own tokens landed (2 arrivals + bytes)
@@ -272,6 +274,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     for (int i = 0; i < L::nbars; ++i) {
       uint32_t cnt = 1;
       if (i >= kLatFull && i < kLatFull + kMlaStages) cnt = 2;
+      if (i == kFinal) cnt = 2;           // the score issuer and the value issuer
       if (i == kPhiFull || i == kPloFull || i == kOFree || i == kSFree || i == kSFree + 1)
         cnt = 2 * kMlaSoftmaxWarps;
       if (i == kQFull) cnt = 2 * kMlaSoftmaxWarps + 2;   // + each CTA's query copy (with its bytes)
@@ -516,8 +519,13 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const uint64_t t0 = globaltimer();
       while (globaltimer() - t0 < 50000) __nanosleep(1000);
     }
-  } else if (warp == kMlaIssuer) {
-    // ------------------------------------------------------------ MMA issuer (rank 0)
+  } else if (warp == kMlaIssuer || warp == kMlaPvIssuer) {
+    // ------------------------------------------------------------ MMA issuers (rank 0)
+    // One thread issues the score MMAs and another the value MMAs, each with its own
+    // commits, so that a tile's value MMA is not queued behind the issue of the next
+    // tile's score MMAs.  The two streams share no tensor or shared memory they
+    // write; every order between them runs through the barriers below.
+    const bool s_role = warp == kMlaIssuer;
     if (rank == 0 && lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, kMlaTile, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16(128, 256, true);
@@ -597,32 +605,33 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           pair::commit_both(&bar[kPhiFree]);
         }
       };
-      // S(m), PVhi(m) and PVlo(m) are each issued in tile order, whichever is ready
-      // first: S(m) once both CTAs' softmax warps have read S(m-2) out of score
-      // buffer m % 2, both CTAs' own tokens of tile m have landed and, at a sequence
-      // start, the query is in place; PVhi(m) once P hi is written and the value
-      // rows are in place in both CTAs and, at a sequence start, the previous O
-      // has been read out; PVlo(m) once P lo is written.
+      // S(m) once both CTAs' softmax warps have read S(m-2) out of score buffer m % 2,
+      // both CTAs' own tokens of tile m have landed and, at a sequence start, the
+      // query is in place.  PVhi(m) once P hi is written and the value rows are in
+      // place in both CTAs and, at a sequence start, the previous O has been read
+      // out; PVlo(m) once P lo is written.  Each stream in tile order.
       int ns = 0, nh = 0, nl = 0;
       uint64_t t_idle = globaltimer();
       uint32_t spins = 0;
-      while (nl < ntiles) {
+      while (s_role ? ns < ntiles : nl < ntiles) {
         bool did = false;
-        if (ns < ntiles &&
-            (ns < 2 || pair::test_cluster(&bar[kSFree + ns % 2], ((ns / 2) & 1) ^ 1)) &&
-            pair::test_cluster(&bar[kLatFull + ns % kMlaStages], (ns / kMlaStages) & 1) &&
-            (!cs.first() || pair::test_cluster(&bar[kQFull], (s_seg + 1) & 1))) {
-          issue_s(ns++);
-          did = true;
-        }
-        if (nh < ns && pair::test_cluster(&bar[kPhiFull], nh & 1) &&
-            (!cp.first() || o_seg < 0 || pair::test_cluster(&bar[kOFree], o_seg & 1))) {
-          issue_pv(nh++, false);
-          did = true;
-        }
-        if (nl < nh && pair::test_cluster(&bar[kPloFull], nl & 1)) {
-          issue_pv(nl++, true);
-          did = true;
+        if (s_role) {
+          if ((ns < 2 || pair::test_cluster(&bar[kSFree + ns % 2], ((ns / 2) & 1) ^ 1)) &&
+              pair::test_cluster(&bar[kLatFull + ns % kMlaStages], (ns / kMlaStages) & 1) &&
+              (!cs.first() || pair::test_cluster(&bar[kQFull], (s_seg + 1) & 1))) {
+            issue_s(ns++);
+            did = true;
+          }
+        } else {
+          if (nh < ntiles && pair::test_cluster(&bar[kPhiFull], nh & 1) &&
+              (!cp.first() || o_seg < 0 || pair::test_cluster(&bar[kOFree], o_seg & 1))) {
+            issue_pv(nh++, false);
+            did = true;
+          }
+          if (nl < nh && pair::test_cluster(&bar[kPloFull], nl & 1)) {
+            issue_pv(nl++, true);
+            did = true;
+          }
         }
         if (did) {
           spins = 0;
@@ -636,8 +645,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         }
       }
     }
-    // every MMA issued has completed before tensor memory is released (an issuer
-    // with nothing to do commits at once)
+    // every MMA issued has completed before tensor memory is released (each issuer
+    // commits once; one with nothing to do commits at once)
     if (rank == 0 && lane == 0) pair::commit_both(&bar[kFinal]);
     __syncwarp();
   } else {
