@@ -592,7 +592,7 @@ pa_status run_mla(int passes, const pa_mla_desc *d, const void *q, const void *l
     mp.lens = cl;
     mp.cap = d->max_blocks_per_seq * d->block_size;
     mp.tile = pa::kMlaTile;
-    mp.seg_units = 0;
+    mp.seg_units = pa::kMlaSeqUnits;
     mp.out = out;
     mp.B = d->batch;
     mp.Hq = pa::kMlaHeads;

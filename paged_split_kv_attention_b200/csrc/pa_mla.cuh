@@ -89,6 +89,10 @@ constexpr int kMlaPvIssuer = 10;          // warp 10: value MMA issue (rank 0)
 constexpr int kMlaThreads = 32 * (kMlaSoftmaxWarps + 3);
 constexpr int kMlaTok = kMlaHalf / 2;     // tokens of a tile per softmax thread
 constexpr int kMlaRescale = 8;            // raise the running max only past 2^8 growth
+#ifndef PA_MLA_SEQ_UNITS
+#define PA_MLA_SEQ_UNITS 3
+#endif
+constexpr int kMlaSeqUnits = PA_MLA_SEQ_UNITS;   // work units counted per sequence besides its tiles
 
 struct MlaParams {
   const uint16_t *q;            // [B][128][576]
@@ -221,16 +225,18 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(sm + L::misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::misc + 4);
   int *scan_scratch = reinterpret_cast<int *>(sm + L::misc + 16);   // [kMlaThreads / 32]
-  int *start = reinterpret_cast<int *>(sm + L::misc + 64);          // b, j of the first tile
+  int *start = reinterpret_cast<int *>(sm + L::misc + 64);          // b, j of the first tile, tiles
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = pair::rank();        // 0: issues the MMAs; heads [64 rank, +64)
   const int pc = blockIdx.x >> 1;            // which piece of the tile stream
   const int cap = p.mbs * p.bs;
 
-  // ---- prologue (all threads): tiles per sequence, block-wide scan, the piece
-  // [tb, te) of the flattened tile stream and the (sequence, tile) it starts at
-  long long tb, te;
+  // ---- prologue (all threads).  The flattened work stream has, for every
+  // non-empty sequence, kMlaSeqUnits empty units (its fixed cost: the query load
+  // and the epilogue, measured at about three tiles' time) and then its tiles.  A
+  // block-wide scan gives the piece [ub, ue) of the stream, the (sequence, tile) of
+  // its first tile and its tile count.
   {
     const int per = (p.B + kMlaThreads - 1) / kMlaThreads;
     const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
@@ -238,7 +244,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     for (int b = b0; b < b1; ++b) {
       const int c = __ldg(&p.context_lens[b]);
       if (blockIdx.x == 0 && (c < 0 || c > cap)) record_error(4 /* PA_ERR_BAD_BLOCK_ID */);
-      local += mla_tiles(c, cap);
+      local += seq_units(c, cap, kMlaTile, kMlaSeqUnits);
     }
     int v = local;
 #pragma unroll
@@ -250,6 +256,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     if (tid == 0) {
       start[0] = 0;
       start[1] = 0;
+      start[2] = 0;
     }
     __syncthreads();
     int run = v - local, total = 0;
@@ -257,18 +264,24 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       if (i < warp) run += scan_scratch[i];
       total += scan_scratch[i];
     }
-    const long long TP = total;
-    const int pieces = used_pieces(p.parts, TP, p.min_tiles, p.B);
-    tb = pc < pieces ? piece_begin(pc, TP, pieces) : 0;
-    te = pc < pieces ? piece_begin(pc + 1, TP, pieces) : 0;
+    const long long TU = total;
+    const int pieces = used_pieces(p.parts, TU, p.min_tiles, p.B);
+    const long long ub = pc < pieces ? piece_begin(pc, TU, pieces) : 0;
+    const long long ue = pc < pieces ? piece_begin(pc + 1, TU, pieces) : 0;
+    int cnt = 0;
     for (int b = b0; b < b1; ++b) {
       const int P = mla_tiles(__ldg(&p.context_lens[b]), cap);
-      if (P > 0 && run <= tb && tb < run + P) {
+      if (P == 0) continue;
+      const long long t0 = run + kMlaSeqUnits, t1 = t0 + P;     // b's tile units
+      if (run <= ub && ub < t1) {               // the sequence holding unit ub
         start[0] = b;
-        start[1] = static_cast<int>(tb - run);
+        start[1] = static_cast<int>(ub > t0 ? ub - t0 : 0);
       }
-      run += P;
+      const long long lo = ub > t0 ? ub : t0, hi = ue < t1 ? ue : t1;
+      if (lo < hi) cnt += static_cast<int>(hi - lo);
+      run += kMlaSeqUnits + P;
     }
+    if (cnt > 0) atomicAdd(&start[2], cnt);
   }
   if (tid == 0) {
     for (int i = 0; i < L::nbars; ++i) {
@@ -303,7 +316,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           reinterpret_cast<uint16_t *>(p.out)[static_cast<long long>(b) * kMlaHeads * kMlaDv + i] = 0;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  const int ntiles = static_cast<int>(te - tb);
+  const int ntiles = start[2];
   const int b_first = start[0], j_first = start[1];
   // the pair barriers, addressed in the rank-0 CTA
   const uint32_t phifull_pair = pair::map_to(&bar[kPhiFull], 0);
