@@ -58,6 +58,8 @@
 // 1 / l, so neither costs anything per token.
 #pragma once
 
+#include <type_traits>
+
 #include "pa_device.cuh"
 #include "pa_merge.cuh"
 
@@ -594,31 +596,54 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
           pl[nt][0] = movmatrix_trans(l01);
           pl[nt][1] = movmatrix_trans(l23);
         }
-        // zero the V^T fragment entries of tokens past the end (stale ring contents)
+        // zero the V^T fragment entries of tokens past the end (stale ring contents);
+        // a full tile skips the masking (the value MMA below, instantiated twice)
         const int tk = 2 * tq;
         const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
         const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
-        // O^T (D x 8NT) += V^T P
-        if (KV8) {
-          // a transposed ldmatrix block (8 tokens x 16 codes read as 8 x 8 pairs)
-          // gives lane (g, tq) the codes of dims 16 c + 2g, 16 c + 2g + 1 for tokens
-          // t0 + 2tq, t0 + 2tq + 1; one byte permute pairs them per dim.  So m-tile
-          // c's fragment rows g and g + 8 are dims 16 c + 2g and 16 c + 2g + 1
-          // (the epilogue writes them there).
+        auto value_mma = [&](auto ragged) {
+          constexpr bool RAGGED = decltype(ragged)::value;
+          // O^T (D x 8NT) += V^T P
+          if (KV8) {
+            // a transposed ldmatrix block (8 tokens x 16 codes read as 8 x 8 pairs)
+            // gives lane (g, tq) the codes of dims 16 c + 2g, 16 c + 2g + 1 for tokens
+            // t0 + 2tq, t0 + 2tq + 1; one byte permute pairs them per dim.  So m-tile
+            // c's fragment rows g and g + 8 are dims 16 c + 2g and 16 c + 2g + 1
+            // (the epilogue writes them there).
 #pragma unroll
-          for (int x = 0; x < KS / 2; ++x) {
-            uint32_t r[4];
-            ldsm_x4_trans(x8_addr(vb, x), r);
+            for (int x = 0; x < KS / 2; ++x) {
+              uint32_t r[4];
+              ldsm_x4_trans(x8_addr(vb, x), r);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int mt = 2 * x + h;
+              for (int h = 0; h < 2; ++h) {
+                const int mt = 2 * x + h;
+                uint32_t a[4];
+                e4m3x4_to_f16x2(__byte_perm(r[2 * h], 0u, 0x3120u), a[0], a[1]);      // tokens 2tq..
+                e4m3x4_to_f16x2(__byte_perm(r[2 * h + 1], 0u, 0x3120u), a[2], a[3]);  // 2tq + 8..
+                if (RAGGED) {
+                  a[0] &= mlo;
+                  a[1] &= mlo;
+                  a[2] &= mhi;
+                  a[3] &= mhi;
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+                  mma_16816<CT>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
               uint32_t a[4];
-              e4m3x4_to_f16x2(__byte_perm(r[2 * h], 0u, 0x3120u), a[0], a[1]);      // tokens 2tq..
-              e4m3x4_to_f16x2(__byte_perm(r[2 * h + 1], 0u, 0x3120u), a[2], a[3]);  // 2tq + 8..
-              a[0] &= mlo;
-              a[1] &= mlo;
-              a[2] &= mhi;
-              a[3] &= mhi;
+              ldsm_x4_trans(vb + sw128_offset(v_row, mt * 16 + v_col, kTile), a);
+              if (RAGGED) {
+                a[0] &= mlo;
+                a[1] &= mlo;
+                a[2] &= mhi;
+                a[3] &= mhi;
+              }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
@@ -626,22 +651,9 @@ gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
               }
             }
           }
-        } else {
-#pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
-            uint32_t a[4];
-            ldsm_x4_trans(vb + sw128_offset(v_row, mt * 16 + v_col, kTile), a);
-            a[0] &= mlo;
-            a[1] &= mlo;
-            a[2] &= mhi;
-            a[3] &= mhi;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              mma_16816<CT>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
-              mma_16816<CT>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
-            }
-          }
-        }
+        };
+        if (ntok < kTile) value_mma(std::true_type{});
+        else value_mma(std::false_type{});
       }
       __syncwarp();              // every lane is done with this stage
       if (!aborted) issue_next();

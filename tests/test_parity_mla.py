@@ -90,6 +90,20 @@ def test_block_sizes(dev, bs):
         assert_close(run(d, inp, num_partitions=parts), ref, f"bs={bs} parts={parts}")
 
 
+def test_piece_bounds_across_sequence_units(dev):
+    # Every non-empty sequence opens the work stream with a few empty units (its
+    # fixed cost) before its tiles, so piece bounds fall before, inside and after
+    # those units, and some pieces hold only empty units.  Many short and long
+    # sequences with explicit piece counts put bounds everywhere.
+    g = np.random.default_rng(11)
+    ctx = [int(x) for x in g.integers(1, 700, 18)] + [0, 96, 97, 191, 192]
+    inp = workloads.make(mla(tuple(ctx), seed=5))
+    ref = ref_of(inp)
+    d = to_dev(inp, dev)
+    for parts in (2, 9, 23, 40, 74, 150):
+        assert_close(run(d, inp, num_partitions=parts), ref, f"parts={parts}")
+
+
 def test_scaled_down_mla_workload(dev):
     inp = workloads.make(workloads.get("mla", batch=3))
     ref = ref_of(inp)
