@@ -344,7 +344,7 @@ cudaError_t merge_dispatch(int DV, bool bf16, const pa::MergeParams &mp, int seg
 // does not cut a short tile stream into pieces much smaller than the partial
 // output each piece writes: a piece leaves G x D fp32 (GQA: one 16-token K+V tile
 // is 16 x D x 4 bytes, so G tiles per piece keep partials at or below the KV
-// bytes read; at least 2) or 128 x 512 fp32 (MLA: 8 tiles of 128 tokens).  A
+// bytes read; at least 2) or 128 x 512 fp32 (MLA: 11 work units of 96-token tiles).  A
 // single short sequence or a single kv head would otherwise spend more on
 // partials and their merge than on the KV.  An explicit partition count is used
 // as given.

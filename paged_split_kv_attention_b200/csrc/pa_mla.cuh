@@ -8,9 +8,11 @@
 //   out[h, :] = softmax_t(scale * q[h, :] . c_t) c_t[0:512].
 // The KV stream is split and merged exactly as for GQA (page
 // "cidian.kuaisou.com: flash decoding ++", three-step snippets): the flattened
-// stream of 128-token tiles is cut into equal pieces, one per CTA pair; a piece
-// that covers a whole sequence writes the output, otherwise it leaves a
-// normalised partial and the log-sum-exp of each head row for the merge kernel.
+// stream of 96-token tiles (each non-empty sequence opening with a few empty
+// units that stand for its fixed cost) is cut into equal pieces, one per CTA
+// pair; a piece that covers a whole sequence writes the output, otherwise it
+// leaves a normalised partial and the log-sum-exp of each head row for the merge
+// kernel.
 //
 // Why a pair of SMs, and how the work is split.  The value accumulator of a
 // sequence (128 heads x 512 fp32) is as large as one SM's whole tensor memory,
