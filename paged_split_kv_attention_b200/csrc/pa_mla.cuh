@@ -92,7 +92,7 @@ constexpr int kMlaThreads = 32 * (kMlaSoftmaxWarps + 3);
 constexpr int kMlaTok = kMlaHalf / 2;     // tokens of a tile per softmax thread
 constexpr int kMlaRescale = 8;            // raise the running max only past 2^8 growth
 #ifndef PA_MLA_SEQ_UNITS
-#define PA_MLA_SEQ_UNITS 3
+#define PA_MLA_SEQ_UNITS 2
 #endif
 constexpr int kMlaSeqUnits = PA_MLA_SEQ_UNITS;   // work units counted per sequence besides its tiles
 
@@ -147,6 +147,14 @@ __device__ __forceinline__ int mla_tiles(int c, int cap) {
 
 // Walks the tiles of a piece in order: sequence b, tile j within it, its tile
 // count P, and whether the tile opens / closes that sequence's run in the piece.
+// 32 bytes from global memory through the non-coherent path (address 32-byte aligned).
+__device__ __forceinline__ void ldg_v8(const void *src, uint32_t *r) {
+  asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "l"(src));
+}
+
 struct MlaCursor {
   const int32_t *cl;
   int B, cap, n, ntiles, b, j, P, ctx;
@@ -236,7 +244,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 
   // ---- prologue (all threads).  The flattened work stream has, for every
   // non-empty sequence, kMlaSeqUnits empty units (its fixed cost: the query load
-  // and the epilogue, measured at about three tiles' time) and then its tiles.  A
+  // and the epilogue, measured at about two tiles' time) and then its tiles.  A
   // block-wide scan gives the piece [ub, ue) of the stream, the (sequence, tile) of
   // its first tile and its tile count.
   {
@@ -696,20 +704,25 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                                       b * kMlaHeads + 64 * static_cast<int>(rank),
                                       kQTmemDims / 64, l2_evict_first_policy());
       }
-      const uint4 *src = reinterpret_cast<const uint4 *>(
-          p.q + (static_cast<long long>(b) * kMlaHeads + head) * kMlaDk);
+      const uint16_t *row = p.q + (static_cast<long long>(b) * kMlaHeads + head) * kMlaDk;
+      // 32-byte loads where the query allows (rows are 1152 bytes apart), else 16
+      const bool wide = (reinterpret_cast<uintptr_t>(p.q) & 31u) == 0;
 #pragma unroll 1
       for (int g = cg == 0 ? 0 : 3; g < (cg == 0 ? 3 : kQTmemDims / 64); ++g) {
-        uint4 x[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = __ldg(src + g * 8 + i);
         uint32_t v[32];
+        if (wide) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[4 * i] = x[i].x;
-          v[4 * i + 1] = x[i].y;
-          v[4 * i + 2] = x[i].z;
-          v[4 * i + 3] = x[i].w;
+          for (int i = 0; i < 4; ++i) ldg_v8(row + g * 64 + 16 * i, v + 8 * i);
+        } else {
+          const uint4 *src = reinterpret_cast<const uint4 *>(row) + g * 8;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 x = __ldg(src + i);
+            v[4 * i] = x.x;
+            v[4 * i + 1] = x.y;
+            v[4 * i + 2] = x.z;
+            v[4 * i + 3] = x.w;
+          }
         }
         tmem_st32u(tmem + kTmQ + g * 32 + lane_off, v);
       }
@@ -918,6 +931,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         const bool whole = n - j >= 0 && n - j + P <= ntiles;
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const long long slot = pc + b;
+        // The rows leave through shared memory: a thread's row would spread each
+        // store instruction over 32 lines.  Warp w stages its 32 rows (TMEM lanes
+        // 32 (w % 4) + r, heads 64 rank + (32 (w % 4) + r) % 64) 64 bytes at a time in
+        // its 2 KB of the P pool, 16-byte chunk k of row r at chunk k ^ ((r >> 1) & 3),
+        // and stores 8 rows x 64 contiguous bytes per instruction.  The pool is free:
+        // the sequence's last value MMA is done, and the next tile's P is written
+        // after the barrier that ends this epilogue.
+        uint8_t *stg = sm + L::ps + warp * 2048;
+        uint8_t *stg_w = stg + lane * 64;
+        const int sw_w = (lane >> 1) & 3;
+        const int rr = lane >> 2, kk = lane & 3;
+        auto stage_row = [&](const uint4 (&w)[4]) {
+          __syncwarp();                                  // the previous pass has been read
+#pragma unroll
+          for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4 *>(stg_w + 16 * (k ^ sw_w)) = w[k];
+          __syncwarp();
+        };
+        auto staged = [&](int i) {                       // row 8 i + rr, chunk kk
+          const int r = 8 * i + rr;
+          return *reinterpret_cast<const uint4 *>(stg + r * 64 + 16 * (kk ^ ((r >> 1) & 3)));
+        };
+        auto head_of = [&](int i) {
+          return 64 * static_cast<int>(rank) + ((32 * (warp & 3) + 8 * i + rr) & 63);
+        };
 #pragma unroll 1
         for (int c = 128 * cg; c < 128 * cg + 128; c += 32) {
           float v[32];
@@ -926,23 +963,37 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           // column c of dims block c / 128: dims 256 (c / 128) + 128 hh + c % 128
           const int d0 = 256 * (c >> 7) + 128 * hh + (c & 127);
           if (whole) {
-            uint16_t *o = reinterpret_cast<uint16_t *>(p.out) +
-                          (static_cast<long long>(b) * kMlaHeads + head) * kMlaDv + d0;
+            uint4 w[4];
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
-              uint4 w;
-              w.x = pack2<true>(v[8 * q8] * inv, v[8 * q8 + 1] * inv);
-              w.y = pack2<true>(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv);
-              w.z = pack2<true>(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv);
-              w.w = pack2<true>(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv);
-              *reinterpret_cast<uint4 *>(o + 8 * q8) = w;
+              w[q8].x = pack2<true>(v[8 * q8] * inv, v[8 * q8 + 1] * inv);
+              w[q8].y = pack2<true>(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv);
+              w[q8].z = pack2<true>(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv);
+              w[q8].w = pack2<true>(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv);
             }
-          } else {
-            float *o = p.part_o + (slot * kMlaHeads + head) * kMlaDv + d0;
+            stage_row(w);
+            uint16_t *o = reinterpret_cast<uint16_t *>(p.out) +
+                          static_cast<long long>(b) * kMlaHeads * kMlaDv + d0 + 8 * kk;
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              *reinterpret_cast<float4 *>(o + 4 * q4) = make_float4(
-                  v[4 * q4] * inv, v[4 * q4 + 1] * inv, v[4 * q4 + 2] * inv, v[4 * q4 + 3] * inv);
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4 *>(o + static_cast<long long>(head_of(i)) * kMlaDv) = staged(i);
+          } else {
+            float *o = p.part_o + slot * kMlaHeads * kMlaDv + d0 + 4 * kk;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint4 w[4];
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const float *x = v + 16 * half + 4 * q4;
+                w[q4] = make_uint4(__float_as_uint(x[0] * inv), __float_as_uint(x[1] * inv),
+                                   __float_as_uint(x[2] * inv), __float_as_uint(x[3] * inv));
+              }
+              stage_row(w);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4 *>(o + static_cast<long long>(head_of(i)) * kMlaDv + 16 * half) =
+                    staged(i);
+            }
           }
         }
         if (!whole && hh == 0 && cg == 0)
@@ -950,6 +1001,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         tc_fence_before();
         __syncwarp();
         if (lane == 0) pair::arrive_remote(ofree_pair);
+        // every softmax warp has read its staged rows before any writes the next P
+        named_bar_sync(3, 32 * kMlaSoftmaxWarps);
       }
     }
   }

@@ -104,6 +104,24 @@ def test_piece_bounds_across_sequence_units(dev):
         assert_close(run(d, inp, num_partitions=parts), ref, f"parts={parts}")
 
 
+def test_query_only_16_byte_aligned(dev):
+    # Query rows are read 32 bytes at a time when the query is 32-byte aligned and
+    # 16 bytes at a time otherwise; a query 16 bytes past an aligned base takes the
+    # second path and must give the same bits.
+    inp = workloads.make(mla((200, 1000, 63), seed=6))
+    ref = ref_of(inp)
+    d = to_dev(inp, dev)
+    q = d["q"]
+    big = torch.empty(q.numel() + 8, dtype=q.dtype, device=dev)
+    q16 = big[8:].view(q.shape)
+    q16.copy_(q)
+    assert q16.data_ptr() % 32 == 16
+    for parts in (0, 3):
+        out = run(dict(d, q=q16), inp, num_partitions=parts)
+        assert_close(out, ref, f"16-byte query parts={parts}")
+        assert torch.equal(out, run(d, inp, num_partitions=parts))
+
+
 def test_scaled_down_mla_workload(dev):
     inp = workloads.make(workloads.get("mla", batch=3))
     ref = ref_of(inp)
