@@ -95,6 +95,13 @@ constexpr int kMlaRescale = 8;            // raise the running max only past 2^8
 #define PA_MLA_SEQ_UNITS 2
 #endif
 constexpr int kMlaSeqUnits = PA_MLA_SEQ_UNITS;   // work units counted per sequence besides its tiles
+#ifndef PA_MLA_PV_FIRST
+#define PA_MLA_PV_FIRST 1
+#endif
+// Tensor-pipe order (1): the score MMA of tile m is issued only after both passes of
+// the value MMA of tile m - 2, so that a tile's value MMA does not queue behind the
+// score MMA of the tile after next (0: each stream issues as soon as it may)
+constexpr bool kMlaPvFirst = PA_MLA_PV_FIRST != 0;
 
 struct MlaParams {
   const uint16_t *q;            // [B][128][576]
@@ -234,6 +241,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   float *xl = xm + 4 * 128;                                        // [2][128] row sums
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(sm + L::misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::misc + 4);
+  volatile int *pv_issued = reinterpret_cast<volatile int *>(sm + L::misc + 8);   // value MMAs issued
   int *scan_scratch = reinterpret_cast<int *>(sm + L::misc + 16);   // [kMlaThreads / 32]
   int *start = reinterpret_cast<int *>(sm + L::misc + 64);          // b, j of the first tile, tiles
 
@@ -304,6 +312,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       mbar_init(&bar[i], cnt);
     }
     *abort_flag = 0;
+    *pv_issued = 0;
     fence_barrier_init();
   }
   if (warp == kMlaIssuer) {
@@ -628,11 +637,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           pair::commit_both(&bar[kPhiFree]);
         }
       };
-      // S(m) once both CTAs' softmax warps have read S(m-2) out of score buffer m % 2,
-      // both CTAs' own tokens of tile m have landed and, at a sequence start, the
-      // query is in place.  PVhi(m) once P hi is written and the value rows are in
-      // place in both CTAs and, at a sequence start, the previous O has been read
-      // out; PVlo(m) once P lo is written.  Each stream in tile order.
+      // S(m) once both CTAs' softmax warps have read S(m-2) out of score buffer
+      // m % 2, both CTAs' own tokens of tile m have landed, at a sequence start the
+      // query is in place, and PVlo(m-2) has been issued.  PVhi(m) once P hi is
+      // written and the value rows are in place in both CTAs and, at a sequence
+      // start, the previous O has been read out; PVlo(m) once P lo is written.  Each
+      // stream in tile order.
       int ns = 0, nh = 0, nl = 0;
       uint64_t t_idle = globaltimer();
       uint32_t spins = 0;
@@ -641,7 +651,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (s_role) {
           if ((ns < 2 || pair::test_cluster(&bar[kSFree + ns % 2], ((ns / 2) & 1) ^ 1)) &&
               pair::test_cluster(&bar[kLatFull + ns % kMlaStages], (ns / kMlaStages) & 1) &&
-              (!cs.first() || pair::test_cluster(&bar[kQFull], (s_seg + 1) & 1))) {
+              (!cs.first() || pair::test_cluster(&bar[kQFull], (s_seg + 1) & 1)) &&
+              (!kMlaPvFirst || ns < 2 || *pv_issued >= ns - 1)) {
             issue_s(ns++);
             did = true;
           }
@@ -653,6 +664,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           }
           if (nl < nh && pair::test_cluster(&bar[kPloFull], nl & 1)) {
             issue_pv(nl++, true);
+            *pv_issued = nl;             // both passes of tile nl - 1 are in the pipe
             did = true;
           }
         }
