@@ -55,12 +55,14 @@
 // online softmax in log2 units (a head's four threads agree on the running max
 // through shared memory, with a lazily raised max), P as bf16 hi + lo (about 16
 // significant bits: a single bf16 copy biases the value mix by up to 2^-9 per
-// weight), zeroing value rows past a ragged end, and the epilogue.  Warp 8
-// issues the TMA loads: its own tokens (completion counted on the rank-0 CTA's
-// barrier, so that the MMA issuer sees both halves land), and, once the tile's
-// scores are done, the other CTA's tokens for its value dims.  Warps 9 and 10 of
-// the rank-0 CTA issue the score and the value MMAs, one thread each.  Every wait
-// is bounded.
+// weight), zeroing value rows past a ragged end, and the epilogue (rows staged
+// through the idle P pool, so that each store instruction covers 8 rows x 64
+// bytes).  Warp 8 issues the TMA loads: its own tokens (completion counted on the
+// rank-0 CTA's barrier, so that the MMA issuer sees both halves land), and, once
+// the tile's scores are done, the other CTA's tokens for its value dims.  Warps 9
+// and 10 of the rank-0 CTA issue the score and the value MMAs, one thread each; a
+// tile's score MMA enters the tensor pipe after the value MMA of the tile two
+// back.  Every wait is bounded.
 #pragma once
 
 #include "pa_device.cuh"
