@@ -65,6 +65,8 @@
 // back.  Every wait is bounded.
 #pragma once
 
+#include <type_traits>
+
 #include "pa_device.cuh"
 #include "pa_tcgen05.cuh"
 
@@ -83,9 +85,11 @@ constexpr int kMlaStages = 3;
 #endif
 constexpr int kMlaLookahead = PA_MLA_LOOKAHEAD;   // own-token tiles issued past the next fetch
 #ifndef PA_MLA_PREFETCH
-#define PA_MLA_PREFETCH 2
+#define PA_MLA_PREFETCH 0
 #endif
-constexpr int kMlaPrefetch = PA_MLA_PREFETCH;     // tiles ahead whose own rows are pulled into L2
+// tiles ahead whose own rows are pulled into L2 (0: none; with the value MMA ahead
+// of the next score MMA in the pipe, a prefetch two tiles ahead cost 6 µs on B64)
+constexpr int kMlaPrefetch = PA_MLA_PREFETCH;
 constexpr int kMlaSoftmaxWarps = 8;       // warps 0-7: softmax and epilogue
 constexpr int kMlaProducer = 8;           // warp 8: copy issue
 constexpr int kMlaIssuer = 9;             // warp 9: score MMA issue (rank 0), TMEM allocation
@@ -709,8 +713,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     // memory with one copy (a 64 dims x 64 rows x 4 slabs box: the 128-byte
     // swizzled K-major layout of the A operand), counted on the rank-0 CTA's
     // query barrier.  Dims [0, 320) go into TMEM lane t as bf16 pairs (both lanes
-    // of the head: the layout of a 2-SM A operand), loaded in five batches of 64
-    // dims.  Called after the previous sequence's last score MMA.
+    // of the head: the layout of a 2-SM A operand), each column group taking half
+    // of them in two batches.  Called after the previous sequence's last score MMA.
     auto load_query = [&](int b) {
       if (t == 0) {
         pair::arrive_expect_tx_remote(qfull_pair, L::kQSlabs * L::kHSlab);
@@ -721,16 +725,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const uint16_t *row = p.q + (static_cast<long long>(b) * kMlaHeads + head) * kMlaDk;
       // 32-byte loads where the query allows (rows are 1152 bytes apart), else 16
       const bool wide = (reinterpret_cast<uintptr_t>(p.q) & 31u) == 0;
-#pragma unroll 1
-      for (int g = cg == 0 ? 0 : 3; g < (cg == 0 ? 3 : kQTmemDims / 64); ++g) {
-        uint32_t v[32];
+      // column group cg writes TMEM columns [80 cg, 80 cg + 80) (dims [160 cg, +160))
+      // in two batches, 32 + 48 columns (cg 0) or 48 + 32 (cg 1), every load of a
+      // batch issued before its stores
+      auto batch = [&](int col, auto ncols_c) {
+        constexpr int NC = decltype(ncols_c)::value;   // 32 or 48
+        uint32_t v[NC];
         if (wide) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) ldg_v8(row + g * 64 + 16 * i, v + 8 * i);
+          for (int i = 0; i < NC / 8; ++i) ldg_v8(row + 2 * col + 16 * i, v + 8 * i);
         } else {
-          const uint4 *src = reinterpret_cast<const uint4 *>(row) + g * 8;
+          const uint4 *src = reinterpret_cast<const uint4 *>(row + 2 * col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < NC / 4; ++i) {
             const uint4 x = __ldg(src + i);
             v[4 * i] = x.x;
             v[4 * i + 1] = x.y;
@@ -738,7 +745,34 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             v[4 * i + 3] = x.w;
           }
         }
-        tmem_st32u(tmem + kTmQ + g * 32 + lane_off, v);
+        auto st32 = [&](int c, int o) {
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = v[o + i];
+          tmem_st32u(tmem + kTmQ + c + lane_off, w);
+        };
+        auto st16 = [&](int c, int o) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = v[o + i];
+          tmem_st16u(tmem + kTmQ + c + lane_off, w);
+        };
+        if constexpr (NC == 32) {
+          st32(col, 0);
+        } else if (col % 32 == 0) {
+          st32(col, 0);
+          st16(col + 32, 32);
+        } else {
+          st16(col, 0);
+          st32(col + 16, 16);
+        }
+      };
+      if (cg == 0) {
+        batch(0, std::integral_constant<int, 32>());
+        batch(32, std::integral_constant<int, 48>());
+      } else {
+        batch(80, std::integral_constant<int, 48>());
+        batch(128, std::integral_constant<int, 32>());
       }
       tmem_wait_st();
       tc_fence_before();
